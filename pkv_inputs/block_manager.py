@@ -1,0 +1,150 @@
+"""Host-side refcounted KV block allocator with copy-on-write.
+
+This is the bookkeeping half of paged KV caching. It decides which physical
+block each logical block of a sequence lives in and which blocks must be copied
+before a write. It moves no KV data: the copies it returns are executed by the
+``kv_block_copy`` kernel (or by the oracle's block copy on the CPU).
+
+What it follows:
+
+* page "PagedAttention Analysis" (ryotta.opik.net), section 2: blocks hold a
+  fixed number B of tokens and are attached on demand. The waste per
+  sequence is therefore at most the unfilled part of its last block (B-1
+  tokens).
+* page "PagedAttention 논문 쉽게 읽기" (iplexlaw.co.kr), section 2: a new
+  token goes into the free slot of the last block, and a fresh block is taken
+  and appended to the table only when that block is full. Section 3 says the
+  same for sharing: a block is shared by reference, a write into a shared block
+  copies it first, and blocks nobody references any more are reclaimed.
+* page "추론 엔진에서의 메모리 가상화" (molayo1419.me), copy-on-write section.
+  Two branches reference blocks #10 and #11 (refcount 2 each). A branch that
+  writes into the partially filled shared block gets a new block (#45). The
+  contents are copied, that branch's table entry is repointed, and the old
+  block's refcount drops by one.
+
+Allocation only updates integer indices on the host. It never touches device
+memory, which matches the pages' point that block management needs no
+``cudaMalloc`` during generation.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class CowCopy:
+    """One whole-block copy ``src -> dst`` that must run before a write."""
+
+    src: int
+    dst: int
+
+
+@dataclass
+class SeqState:
+    """A sequence's block table (logical -> physical) and its token count."""
+
+    table: List[int] = field(default_factory=list)
+    num_tokens: int = 0
+
+
+class BlockAllocator:
+    """Free list plus a refcount per physical block.
+
+    ``free_order`` fixes the order in which free blocks are handed out. A
+    seeded permutation of ``range(num_blocks)`` scatters sequences over the
+    pool, and an explicit list reproduces a worked example.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int,
+                 free_order: Optional[Sequence[int]] = None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise ValueError("num_blocks and block_size must be positive")
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+        order = list(range(num_blocks)) if free_order is None else [int(b) for b in free_order]
+        listed = set(order)
+        if len(listed) != len(order) or any(b < 0 or b >= num_blocks for b in order):
+            raise ValueError("free_order must list distinct block ids in [0, num_blocks)")
+        # pop() takes from the end, so store the order reversed
+        self._free: List[int] = order[::-1]
+        self._ref = np.zeros(num_blocks, dtype=np.int64)
+        for b in range(num_blocks):
+            if b not in listed:
+                self._ref[b] = 1 << 40  # never handed out
+        self.copies: List[CowCopy] = []
+
+    # -- primitive operations -------------------------------------------------
+    @property
+    def num_free(self) -> int:
+        return len(self._free)
+
+    def refcount(self, block: int) -> int:
+        return int(self._ref[block])
+
+    def allocate(self) -> int:
+        if not self._free:
+            raise MemoryError("KV block pool exhausted")
+        b = self._free.pop()
+        assert self._ref[b] == 0
+        self._ref[b] = 1
+        return b
+
+    def free(self, block: int) -> None:
+        if self._ref[block] <= 0:
+            raise ValueError(f"block {block} freed more often than referenced")
+        self._ref[block] -= 1
+        if self._ref[block] == 0:
+            self._free.append(block)
+
+    # -- sequence-level operations -------------------------------------------
+    def new_sequence(self, num_tokens: int) -> SeqState:
+        """Attach ceil(num_tokens / B) fresh blocks for a prompt."""
+        seq = SeqState()
+        nb = -(-int(num_tokens) // self.block_size)
+        seq.table = [self.allocate() for _ in range(nb)]
+        seq.num_tokens = int(num_tokens)
+        return seq
+
+    def fork(self, seq: SeqState) -> SeqState:
+        """A new sequence that shares every block of ``seq`` by reference."""
+        for b in seq.table:
+            self._ref[b] += 1
+        return SeqState(table=list(seq.table), num_tokens=seq.num_tokens)
+
+    def append_slot(self, seq: SeqState) -> Tuple[int, Optional[CowCopy]]:
+        """Reserve the slot for the sequence's next token.
+
+        Returns ``(slot, copy)`` where ``slot = phys_block * B + offset`` and
+        ``copy`` is the copy-on-write that must run first, or ``None``.
+        """
+        B = self.block_size
+        off = seq.num_tokens % B
+        cow = None
+        if off == 0:
+            seq.table.append(self.allocate())
+        else:
+            last = seq.table[-1]
+            if self._ref[last] > 1:
+                new = self.allocate()
+                cow = CowCopy(src=last, dst=new)
+                self._ref[last] -= 1
+                seq.table[-1] = new
+                self.copies.append(cow)
+        slot = seq.table[-1] * B + off
+        seq.num_tokens += 1
+        return slot, cow
+
+    def release(self, seq: SeqState) -> None:
+        for b in seq.table:
+            self.free(b)
+        seq.table = []
+        seq.num_tokens = 0
+
+    @staticmethod
+    def waste_slots(seq: SeqState, block_size: int) -> int:
+        """Reserved but unfilled slots of a sequence (its last block only)."""
+        return len(seq.table) * block_size - seq.num_tokens

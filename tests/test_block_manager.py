@@ -1,0 +1,103 @@
+"""Host block allocator: the pages' copy-on-write example, the waste bound
+and the byte-count helper, each against a cited golden fixture."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from pkv_inputs import BlockAllocator, kv_bytes_per_token, make_shared_prefix_case
+from pkv_inputs.block_manager import SeqState
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def test_cow_worked_example():
+    g = load("cow_worked_example.json")
+    B, P = g["block_size"], g["num_blocks"]
+    others = [b for b in range(P) if b not in g["prompt_blocks"] + [g["next_free_block"]]]
+    order = g["prompt_blocks"] + [g["next_free_block"]] + others
+    alloc = BlockAllocator(P, B, free_order=order)
+    a = alloc.new_sequence(g["prompt_tokens"])
+    assert a.table == g["prompt_blocks"]
+    b = alloc.fork(a)
+    assert [alloc.refcount(x) for x in a.table] == [2, 2]
+    exp = g["expected"]
+    slot, cow = alloc.append_slot(a)
+    assert (cow.src, cow.dst) == tuple(exp["copy"])
+    assert a.table == exp["branch_a_table"]
+    assert b.table == exp["branch_b_table"]
+    assert slot == exp["branch_a_slot"]
+    for blk, ref in exp["refcounts"].items():
+        assert alloc.refcount(int(blk)) == ref
+    # branch B is now the only owner of block 11 and writes in place
+    slot_b, cow_b = alloc.append_slot(b)
+    assert cow_b is exp["branch_b_copy_on_its_write"]
+    assert slot_b == 11 * B + g["prompt_tokens"] % B
+
+
+def test_waste_bounded_by_last_block():
+    g = load("block_waste.json")
+    B = g["block_size"]
+    rng = np.random.default_rng(0)
+    alloc = BlockAllocator(100000, B, free_order=rng.permutation(100000).tolist())
+    wastes = []
+    for L in rng.integers(1, 5000, size=2000):
+        s = alloc.new_sequence(int(L))
+        w = BlockAllocator.waste_slots(s, B)
+        assert 0 <= w <= g["max_waste_tokens"]
+        wastes.append(w)
+        alloc.release(s)
+    assert abs(np.mean(wastes) - g["mean_waste_tokens_uniform_lengths"]) < 0.5
+
+
+def test_growth_allocates_only_when_last_block_full():
+    alloc = BlockAllocator(8, 4)
+    s = alloc.new_sequence(3)
+    assert len(s.table) == 1
+    slot, cow = alloc.append_slot(s)      # fills the 4th slot
+    assert cow is None and len(s.table) == 1 and slot == s.table[0] * 4 + 3
+    slot, cow = alloc.append_slot(s)      # block full -> new block
+    assert cow is None and len(s.table) == 2 and slot == s.table[1] * 4
+
+
+def test_release_returns_blocks_when_unreferenced():
+    alloc = BlockAllocator(6, 16)
+    a = alloc.new_sequence(20)
+    b = alloc.fork(a)
+    free0 = alloc.num_free
+    alloc.release(a)
+    assert alloc.num_free == free0           # still referenced by b
+    alloc.release(b)
+    assert alloc.num_free == 6
+    with pytest.raises(ValueError):
+        alloc.free(0)
+
+
+def test_opt13b_bytes_per_token():
+    g = load("opt13b_kv_bytes.json")
+    n = kv_bytes_per_token(g["num_layers"], g["num_kv_heads"], g["head_dim"], g["elem_bytes"])
+    assert n == g["expected_bytes_per_token"]
+    assert n / 1024 == g["expected_kib_per_token"]
+    lo, hi = g["expected_max_sequence_gb_range"]
+    assert lo <= n * g["max_positions"] / 1e9 <= hi
+
+
+def test_shared_prefix_copies_follow_refcount_rule():
+    c = make_shared_prefix_case(num_prompts=2, samples=3, prompt_len=40, decode_steps=5,
+                                num_heads=2, num_kv_heads=2, head_dim=64)
+    # per prompt: samples-1 copies (the last writer owns the block alone)
+    assert c.cow_pairs.shape == (2 * 2, 2)
+    assert len(set(c.cow_pairs[:, 1].tolist())) == 4
+    st = c.steps[-1]
+    assert st["context_lens"].tolist() == [45] * 6
+    # full prompt blocks stay shared across the samples of one prompt
+    bt = st["block_tables"]
+    assert (bt[0, :2] == bt[1, :2]).all() and (bt[0, :2] == bt[2, :2]).all()
+    assert bt[0, 2] != bt[1, 2] != bt[2, 2]
