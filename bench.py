@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark: paged decode attention on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one batch:
+``kv_cache_append`` of every sequence's newest token (through its slot
+mapping), then ``paged_attn_decode`` over all cached tokens. The decode
+includes the split-context merge when a context exceeds one partition. The
+default workload is the Llama-8B-shaped GQA batch:
+
+  * 256 sequences, 32 query heads / 8 KV heads, head_dim 128, bf16
+  * 16-token blocks, lognormal context lengths (median 512, capped at 4096)
+  * shuffled physical blocks
+
+Copy-on-write block copies happen only on forks; the shared-prefix workload
+(``--workload shared_prefix``) includes them.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own batch: weak scaling, no data collective.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: effective KV GB/s (% of HBM peak), seq-steps/s"
+HBM_SPEC_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ("paged_kv_cache_387_b200/csrc/decode_tc.cu",
+                  "paged_kv_cache_387_b200/csrc/pkv_device.cuh")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_gqa_b256")
+    ap.add_argument("--soak-seconds", type=float, default=2.0,
+                    help="back-to-back steps before the timed region (clock sampling, warm clocks)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--contiguous", action="store_true",
+                    help="also time the same batch with identity block placement")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"decode_tc_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.strip().startswith(("source_sha256", "traffic_bytes_per_launch")):
+                k, v = line.strip().split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    try:
+        if vals.get("source_sha256") == decode_source_hash():
+            return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples (timestamps on the host clock)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.samples = []
+        self.proc = None
+        self.gpu_index = gpu_index
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1, window):
+        sel = [p for (t, p) in self.samples if t0 <= t <= t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window": window}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(p[1]) for p in sel if num(p[1]) is not None]
+        smax = [num(p[2]) for p in sel if num(p[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in sel:
+            for name, v in zip(names, p[5:9]):
+                if v.strip().lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sel), "window": window,
+                "power_w_max": max((num(p[3]) or 0.0) for p in sel)}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the CPU oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(case_cpu, nseq):
+    """One oracle step (append + decode) over the first ``nseq`` sequences."""
+    import torch
+    import oracle
+    sl = slice(0, nseq)
+    if case_cpu.slot_mapping is not None:
+        oracle.cache_append(case_cpu.k_pool, case_cpu.v_pool, case_cpu.k_new[sl].contiguous(),
+                            case_cpu.v_new[sl].contiguous(),
+                            case_cpu.slot_mapping[sl].contiguous())
+    oracle.paged_decode(case_cpu.q[sl].contiguous(), case_cpu.k_pool, case_cpu.v_pool,
+                        case_cpu.block_tables[sl].contiguous(),
+                        case_cpu.context_lens[sl].contiguous(), case_cpu.scale)
+
+
+def size_oracle_sample(case_cpu, target_s):
+    """Pick the number of leading sequences whose oracle step takes about target_s."""
+    n = 1
+    t = 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle_sample_step(case_cpu, n)
+        t = time.perf_counter() - t0
+        if t >= 0.05 * target_s or n >= case_cpu.num_seqs:
+            break
+        n = min(case_cpu.num_seqs, n * 4)
+    est = max(1, int(n * target_s / max(t, 1e-6)))
+    return min(case_cpu.num_seqs, est)
+
+
+def step_bytes(case, nseq=None):
+    """Algorithmic bytes of one step (decode + the append that precedes it)."""
+    from pkv_inputs import decode_algorithmic_bytes
+    lens = case.context_lens.cpu().tolist()
+    if nseq is not None:
+        lens = lens[:nseq]
+    es = case.q.element_size()
+    b = decode_algorithmic_bytes(lens, case.num_heads, case.num_kv_heads, case.head_dim,
+                                 case.block_size, es)
+    app = 0
+    if case.slot_mapping is not None:
+        t = len(lens)
+        # read new K and V + slot, write them into the pool
+        app = t * (2 * 2 * case.num_kv_heads * case.head_dim * es + 8)
+    return b, app
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import torch
+    import oracle
+    from pkv_inputs import make_case
+    oracle.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    case = make_case(args.workload, device=dev, with_append=True).to("cpu")
+    budget = 150.0  # seconds for warmup + steps
+    per_step = min(2.0, budget / max(1, args.steps + args.warmup))
+    nseq = size_oracle_sample(case, per_step)
+    for _ in range(args.warmup):
+        oracle_sample_step(case, nseq)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(case, nseq)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    dec, app = step_bytes(case, nseq)
+    gbs = (dec + app) / dt / 1e9
+    sample = (f"first {nseq} of {case.num_seqs} sequences "
+              f"({int(case.context_lens[:nseq].sum())} tokens), append + decode, fp64 oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(case, args.workload, args.gpus),
+        "seq_steps_per_s": nseq / dt,
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+def config_block(case, workload, n_gpus):
+    from pkv_inputs.workloads import WORKLOADS
+    desc = WORKLOADS.get(workload, {}).get("desc", workload)
+    return {
+        "workload": workload, "desc": desc, "num_seqs_per_gpu": case.num_seqs,
+        "num_heads": case.num_heads, "num_kv_heads": case.num_kv_heads,
+        "head_dim": case.head_dim, "block_size": case.block_size,
+        "partition_size": case.partition_size,
+        "context_tokens_per_gpu": int(case.context_lens.sum()),
+        "max_context_len": case.max_context_len,
+        "step": "kv_cache_append (newest token of each sequence) + paged_attn_decode",
+        "accumulate": "fp32",
+        "l2": "inputs larger than L2: the K/V pool read each step is "
+              f"{case.k_pool.numel() * case.k_pool.element_size() * 2 / 1e9:.2f} GB per GPU",
+        "parallelism": f"{n_gpus} independent batches, one per GPU (no data collective)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import paged_kv_cache_387_b200 as pkv
+    from paged_kv_cache_387_b200 import build as pkv_build
+    from pkv_inputs import make_case
+
+    if rank == 0 or not os.path.exists(pkv.LIB_PATH):
+        pkv_build.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    case = make_case(args.workload, device=dev, with_append=True)
+    stream = torch.cuda.current_stream(dev)
+
+    S, Hq, D = case.num_seqs, case.num_heads, case.head_dim
+    mcl = case.max_context_len
+    out = torch.empty_like(case.q)
+    ws_bytes = pkv.decode_workspace_bytes(S, Hq, D, mcl, case.partition_size)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    launches_per_step = 1 + 1 + (1 if ws_bytes > 0 else 0)
+
+    def decode(c, o):
+        pkv.paged_attn_decode(o, c.q, c.k_pool, c.v_pool, c.block_tables, c.context_lens,
+                              c.scale, mcl, partition_size=c.partition_size, workspace=ws,
+                              err=err)
+
+    def step(ev_pair=None):
+        pkv.kv_cache_append(case.k_pool, case.v_pool, case.k_new, case.v_new,
+                            case.slot_mapping, err=err)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        decode(case, out)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else local_rank)
+    if rank == 0:
+        sampler.start()
+    t_soak0 = time.time()
+    # soak: back-to-back steps so clocks settle and samples exist next to the timed region
+    while time.time() - t_soak0 < args.soak_seconds:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
+
+    dec_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        step(dec_events[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_host1 = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+
+    ms = start.elapsed_time(end) / args.steps
+    dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_events)
+    if world > 1:
+        t = torch.tensor([ms, dec_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(t[0]), float(t[1])
+
+    dec_bytes, app_bytes = step_bytes(case)
+    total_bytes = (dec_bytes + app_bytes) * world
+    value = total_bytes / (ms * 1e-3) / 1e9
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    host_in = {k: getattr(case, k).cpu().pin_memory()
+               for k in ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")}
+    dev_in = {k: getattr(case, k) for k in host_in}
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
+
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word set: {pkv.device_error_message(int(err.item()))}")
+
+    contiguous = None
+    if args.contiguous:
+        ccase = make_case(args.workload, device=dev, with_append=False, placement="identity")
+        cout = torch.empty_like(ccase.q)
+        for _ in range(3):
+            decode(ccase, cout)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            decode(ccase, cout)
+        b.record(stream)
+        torch.cuda.synchronize()
+        cms = a.elapsed_time(b) / args.steps
+        contiguous = {"decode_ms_identity_placement": cms, "decode_ms_shuffled": dec_ms,
+                      "paged_over_contiguous_time": dec_ms / cms}
+        del ccase, cout
+
+    if rank != 0:
+        return None
+
+    peak, peak_kind = measured_peaks()
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(args.workload)
+    clocks = sampler.summary(t_soak0, t_host1,
+                             "soak + timed region" if t_host1 - t_host0 < 1.0 else "timed region")
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": str(case.q.dtype).replace("torch.", "").replace("bfloat16", "bf16")
+                 .replace("float16", "f16").replace("float32", "f32"),
+        "data": "synthetic",
+        "config": config_block(case, args.workload, world),
+        "seq_steps_per_s": S * world / (ms * 1e-3),
+        "pct_of_hbm_peak": {"of_spec_8000_gbs": value / (HBM_SPEC_GBS * world),
+                            f"of_{peak_kind}_{peak:.0f}_gbs": value / (peak * world)},
+        "roofline": {"kernel": "paged_attn_decode (decode_tc_kernel + merge_kernel)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": dec_bytes,
+                     "decode_ms": dec_ms},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if contiguous:
+        line["paged_vs_contiguous"] = contiguous
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, args.cpu_seconds)
+    return line
+
+
+def cpu_baseline(case, target_s):
+    import oracle
+    oracle.build()
+    c = case.to("cpu")
+    nseq = size_oracle_sample(c, target_s)
+    t0 = time.perf_counter()
+    oracle_sample_step(c, nseq)
+    dt = time.perf_counter() - t0
+    dec, app = step_bytes(c, nseq)
+    return {"value": (dec + app) / dt / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {nseq} of {c.num_seqs} sequences "
+                      f"({int(c.context_lens[:nseq].sum())} tokens), one append + decode step, "
+                      f"{dt:.1f} s"}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * pkv.h - C ABI of the paged KV-cache decode library (sm_100a).
+ *
+ * Three operations on a KV cache split into fixed-size blocks that sit
+ * non-contiguously in one physical pool per K and V:
+ *
+ *   paged_attn_decode  single-query attention of every sequence over its
+ *                      cached tokens, read through its block table
+ *   kv_cache_append    scatter new tokens' K/V into their pool slots
+ *   kv_block_copy      whole-block copies (copy-on-write of shared blocks)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers. Every data pointer is a DEVICE pointer owned by the caller. The
+ * library never allocates, frees or retains memory. Block allocation is host
+ * bookkeeping over integer block ids, and needs no device allocation during
+ * generation (page "추론 엔진에서의 메모리 가상화", molayo1419.me, block
+ * manager section).
+ *
+ * Streams. `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ * default stream. Work is enqueued on it and the call returns without
+ * synchronising.
+ *
+ * Element types. pkv_dtype gives the element type of q, out and both pools.
+ *
+ * Pool layout. Both pools are [num_blocks][num_kv_heads][block_size][head_dim],
+ * row-major, head_dim contiguous. Token t of a sequence with block table bt
+ * is at block bt[t / block_size], slot t % block_size. One (block, kv head)
+ * slice is block_size*head_dim contiguous elements.
+ *
+ * Errors. Argument errors that the host can check return PKV_EINVAL or
+ * PKV_EUNSUPPORTED synchronously, with nothing enqueued. A failed launch
+ * returns PKV_ECUDA. Conditions only the device can see (a block id outside
+ * [0, num_blocks), a slot beyond the pool, a context length above
+ * max_context_len) never fault. The offending access is skipped (its tokens
+ * are masked), and if `err` is non-NULL the first such condition's
+ * PKV_DEV_* code is stored there with an atomic compare-and-swap from 0.
+ * The caller zeroes *err and reads it after the stream completes.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_EINVAL = -1,       /* bad argument (null pointer, negative size, misalignment...) */
+  PKV_EUNSUPPORTED = -2, /* valid but not implemented (head_dim, block_size, group size) */
+  PKV_ECUDA = -3,        /* a CUDA runtime call or launch failed */
+} pkv_status;
+
+typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+/* Device-side error codes stored into *err (first one wins). */
+enum {
+  PKV_DEV_BAD_BLOCK = 1,     /* block-table entry outside [0, num_blocks) */
+  PKV_DEV_BAD_SLOT = 2,      /* append slot >= num_blocks * block_size */
+  PKV_DEV_BAD_PAIR = 3,      /* copy pair with src or dst outside [0, num_blocks) */
+  PKV_DEV_CONTEXT_LEN = 4,   /* context_lens[s] > max_context_len or > table capacity */
+  PKV_DEV_WAIT_TIMEOUT = 5,  /* an on-chip copy wait gave up (never expected) */
+};
+
+/*
+ * Bytes of device workspace paged_attn_decode needs for these sizes. The
+ * answer is 0 when no sequence needs more than one partition. This function
+ * is pure arithmetic: it does not touch the GPU.
+ */
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
+                                  int max_context_len, int partition_size);
+
+/*
+ * paged_attn_decode - one decode step of attention over a paged KV cache.
+ *
+ * For every sequence s and query head h, with G = num_heads / num_kv_heads,
+ * g = h / G and L = context_lens[s]:
+ *   o[s][h] = sum_{t<L} softmax_t(scale * q[s][h] . k_t) * v_t
+ * where k_t and v_t are token t's vectors of KV head g, found through
+ * block_tables[s]. This is the causal attention of the newest token over all
+ * L cached tokens, which includes itself (page "PagedAttention", newikis,
+ * section "Mathematical formulation": causal attention, and its block-wise
+ * form, which is identical in value). Scores are taken block by block with a
+ * running max and sum. That is the online-softmax walk over the block table
+ * in page "PagedAttention Analysis" (ryotta.opik.net), section 3.
+ * Accumulation is fp32. The output is rounded to the input type
+ * (round-to-nearest-even).
+ *
+ * Long contexts are split into partitions of partition_size tokens. Each
+ * partition is attended independently, and the partials are combined by
+ * log-sum-exp weights.
+ *
+ * out            [num_seqs][num_heads][head_dim], written entirely. A sequence
+ *                with L <= 0 gets zeros.
+ * q              [num_seqs][num_heads][head_dim]
+ * k_pool, v_pool [num_blocks][num_kv_heads][block_size][head_dim]. Must be
+ *                16-byte aligned.
+ * block_tables   int32 [num_seqs][max_blocks_per_seq], physical block ids.
+ *                Entries at or beyond ceil(L / block_size) are never read.
+ * context_lens   int32 [num_seqs]. Precondition: 0 <= L <= max_context_len,
+ *                and ceil(L / block_size) <= max_blocks_per_seq.
+ * max_context_len a host-side upper bound on context_lens. It sizes the
+ *                grid and the workspace, so the call needs no device-to-host read.
+ * scale          score multiplier; 1/sqrt(head_dim) gives the usual attention.
+ * partition_size tokens per partition. 0 means no split (one partition of
+ *                the whole context). Otherwise a positive multiple of 16.
+ * workspace      device scratch of at least pkv_decode_workspace_bytes(...)
+ *                bytes, 16-byte aligned. It may be NULL when that size is 0.
+ *                Its contents on entry do not matter.
+ * err            nullable device int32 error word (see above).
+ *
+ * Supported: head_dim in {64, 128}; f32 with any block_size >= 1; f16/bf16
+ * with block_size a multiple of 16 (up to 256) and num_heads/num_kv_heads <= 8.
+ * Anything else returns PKV_EUNSUPPORTED.
+ */
+int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
+                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                      int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                      int32_t *err, void *stream);
+
+/*
+ * kv_cache_append - write new tokens' K/V into their slots.
+ *
+ * For each token i < num_tokens with slot = slot_mapping[i] >= 0 and every KV
+ * head h:
+ *   k_pool[slot / block_size][h][slot % block_size][:] = k_new[i][h][:]
+ *   v_pool[slot / block_size][h][slot % block_size][:] = v_new[i][h][:]
+ * A new token goes into the free slot of its sequence's last block (page
+ * "PagedAttention 논문 쉽게 읽기", iplexlaw.co.kr, section 2). Negative slots are
+ * skipped. A slot >= num_blocks*block_size is skipped and reported in *err.
+ * The copy is bit-exact.
+ *
+ * k_new, v_new  [num_tokens][num_kv_heads][head_dim], 16-byte aligned.
+ * slot_mapping  int64 [num_tokens]. Precondition: the non-negative slots are
+ *               distinct. Otherwise which token lands in a repeated slot is
+ *               unspecified.
+ */
+int kv_cache_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,
+                    const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                    int head_dim, int block_size, int num_blocks, int dtype, int32_t *err,
+                    void *stream);
+
+/*
+ * kv_block_copy - copy whole physical blocks, as copy-on-write requires.
+ *
+ * For each pair i < num_pairs, (src, dst) = (src_dst[2i], src_dst[2i+1]), all
+ * num_kv_heads*block_size*head_dim elements of block src are copied to block
+ * dst, in both pools. A write into a block whose refcount is above one copies
+ * the block first (page "추론 엔진에서의 메모리 가상화", molayo1419.me,
+ * copy-on-write section: old block #11 copied into new block #45). The copy
+ * is bit-exact.
+ *
+ * src_dst  device int32 [num_pairs][2]. Precondition: the dst blocks are
+ *          distinct, and no dst is also a src in the same call. Pairs run
+ *          concurrently. A pair with an id outside [0, num_blocks) is
+ *          skipped and reported in *err.
+ */
+int kv_block_copy(void *k_pool, void *v_pool, const int32_t *src_dst, int num_pairs,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                  int32_t *err, void *stream);
+
+/* Static, human-readable text for a pkv_status value. */
+const char *pkv_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,177 @@
+"""Python binding of the paged KV-cache decode library (``libpkv.so``).
+
+The functions below only marshal arguments: they check torch tensors' devices,
+dtypes, shapes and contiguity, pass their device pointers and the current CUDA
+stream to the C ABI declared in ``include/pkv.h``, and raise on a non-zero
+status. Every step of the computation runs in the library's CUDA kernels;
+there is no fallback path. If the library is not built, every call raises.
+
+Pool layout: ``[num_blocks][num_kv_heads][block_size][head_dim]``, head_dim
+contiguous; token t of a sequence is at block ``block_tables[s][t // B]``,
+slot ``t % B``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpkv.so")
+
+PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ECUDA = 0, -1, -2, -3
+DEV_ERRORS = {1: "block id out of range", 2: "append slot out of range",
+              3: "copy pair out of range", 4: "context length above max_context_len",
+              5: "copy wait timed out"}
+DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+DEFAULT_PARTITION = 512
+
+EXPORTS = ("paged_attn_decode", "kv_cache_append", "kv_block_copy",
+           "pkv_decode_workspace_bytes", "pkv_status_string")
+
+
+class PkvError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library():
+    """Load ``libpkv.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"CUDA library not built: {LIB_PATH} is missing "
+            "(run `python paged_kv_cache_387_b200/build.py`)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.paged_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, Z, P, P]
+    lib.paged_attn_decode.restype = I
+    lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
+    lib.kv_cache_append.restype = I
+    lib.kv_block_copy.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
+    lib.kv_block_copy.restype = I
+    lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.pkv_decode_workspace_bytes.restype = Z
+    lib.pkv_status_string.argtypes = [I]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, rc: int):
+    if rc != PKV_OK:
+        msg = load_library().pkv_status_string(rc).decode()
+        raise PkvError(fn, rc, msg)
+
+
+def _dev_ptr(t: Optional[torch.Tensor], name: str, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int, max_context_len: int,
+                           partition_size: int = DEFAULT_PARTITION) -> int:
+    return int(load_library().pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
+                                                         max_context_len, partition_size))
+
+
+def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
+                      v_pool: torch.Tensor, block_tables: torch.Tensor,
+                      context_lens: torch.Tensor, scale: float, max_context_len: int,
+                      partition_size: int = DEFAULT_PARTITION,
+                      workspace: Optional[torch.Tensor] = None,
+                      err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step of paged attention; writes ``out`` [S][Hq][D]."""
+    lib = load_library()
+    dev = q.device
+    if q.dtype not in DTYPE_CODES or out.dtype != q.dtype or k_pool.dtype != q.dtype \
+            or v_pool.dtype != q.dtype:
+        raise TypeError("q, out, k_pool and v_pool must share one of float32/float16/bfloat16")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    S, Hq, D = (int(x) for x in q.shape)
+    P, Hkv, B, D2 = (int(x) for x in k_pool.shape)
+    if tuple(out.shape) != (S, Hq, D) or tuple(v_pool.shape) != (P, Hkv, B, D2) or D2 != D:
+        raise ValueError("shape mismatch between q/out/k_pool/v_pool")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [S][max_blocks] and context_lens [S]")
+    need = decode_workspace_bytes(S, Hq, D, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.paged_attn_decode(
+        _dev_ptr(out, "out", dev), _dev_ptr(q, "q", dev), _dev_ptr(k_pool, "k_pool", dev),
+        _dev_ptr(v_pool, "v_pool", dev), _dev_ptr(block_tables, "block_tables", dev),
+        _dev_ptr(context_lens, "context_lens", dev), S, Hq, Hkv, D, B,
+        int(block_tables.shape[1]), P, int(max_context_len), float(scale), DTYPE_CODES[q.dtype],
+        int(partition_size), _dev_ptr(workspace, "workspace", dev), ws_bytes,
+        _dev_ptr(err, "err", dev), _stream_ptr(stream, dev))
+    _check("paged_attn_decode", rc)
+    return out
+
+
+def kv_cache_append(k_pool: torch.Tensor, v_pool: torch.Tensor, k_new: torch.Tensor,
+                    v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                    err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Scatter ``k_new``/``v_new`` [T][Hkv][D] into pool slots ``slot_mapping`` (int64 [T])."""
+    lib = load_library()
+    dev = k_pool.device
+    if k_pool.dtype not in DTYPE_CODES or any(t.dtype != k_pool.dtype
+                                              for t in (v_pool, k_new, v_new)):
+        raise TypeError("pools and new tokens must share one of float32/float16/bfloat16")
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    P, Hkv, B, D = (int(x) for x in k_pool.shape)
+    T = int(slot_mapping.shape[0])
+    if tuple(k_new.shape) != (T, Hkv, D) or tuple(v_new.shape) != (T, Hkv, D) \
+            or tuple(v_pool.shape) != (P, Hkv, B, D):
+        raise ValueError("shape mismatch between pools, new tokens and slot_mapping")
+    rc = lib.kv_cache_append(_dev_ptr(k_pool, "k_pool", dev), _dev_ptr(v_pool, "v_pool", dev),
+                             _dev_ptr(k_new, "k_new", dev), _dev_ptr(v_new, "v_new", dev),
+                             _dev_ptr(slot_mapping, "slot_mapping", dev), T, Hkv, D, B, P,
+                             DTYPE_CODES[k_pool.dtype], _dev_ptr(err, "err", dev),
+                             _stream_ptr(stream, dev))
+    _check("kv_cache_append", rc)
+
+
+def kv_block_copy(k_pool: torch.Tensor, v_pool: torch.Tensor, src_dst: torch.Tensor,
+                  err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Copy whole blocks ``src_dst[i] = (src, dst)`` (int32 [N][2]) in both pools."""
+    lib = load_library()
+    dev = k_pool.device
+    if k_pool.dtype not in DTYPE_CODES or v_pool.dtype != k_pool.dtype:
+        raise TypeError("pools must share one of float32/float16/bfloat16")
+    if src_dst.dtype != torch.int32 or (src_dst.numel() and src_dst.dim() != 2):
+        raise TypeError("src_dst must be int32 [N][2]")
+    P, Hkv, B, D = (int(x) for x in k_pool.shape)
+    N = int(src_dst.shape[0]) if src_dst.numel() else 0
+    rc = lib.kv_block_copy(_dev_ptr(k_pool, "k_pool", dev), _dev_ptr(v_pool, "v_pool", dev),
+                           _dev_ptr(src_dst, "src_dst", dev) if N else None, N, Hkv, D, B, P,
+                           DTYPE_CODES[k_pool.dtype], _dev_ptr(err, "err", dev),
+                           _stream_ptr(stream, dev))
+    _check("kv_block_copy", rc)
+
+
+def device_error_message(code: int) -> str:
+    return DEV_ERRORS.get(int(code), f"code {int(code)}")

@@ -1,0 +1,211 @@
+// C ABI entry points: argument checks, workspace layout, TMA descriptors and
+// launches. No allocation happens here. Every buffer belongs to the caller.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "pkv.h"
+#include "pkv_internal.h"
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Partitions needed for the longest allowed context (1 when unsplit).
+long long parts_for(int max_context_len, int partition_size) {
+  if (partition_size <= 0) return 1;
+  const long long L = max_context_len > 0 ? max_context_len : 1;
+  return (L + partition_size - 1) / partition_size;
+}
+
+// Workspace = [S][Hq][max_parts][D] float partials, then [S][Hq][max_parts]
+// float log2-sum-exp values, each region 256-byte aligned.
+size_t workspace_layout(long long S, long long Hq, long long D, long long max_parts,
+                        size_t *lse_offset) {
+  const size_t o_bytes = round_up((size_t)(S * Hq * max_parts * D) * sizeof(float), 256);
+  const size_t l_bytes = round_up((size_t)(S * Hq * max_parts) * sizeof(float), 256);
+  *lse_offset = o_bytes;
+  return o_bytes + l_bytes;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A pool viewed as a 2-D tensor [rows = num_blocks*Hkv*B][D] of 16-bit
+// elements. It is read in boxes of 64 elements x 16 rows under the 128-byte
+// swizzle.
+bool make_pool_map(CUtensorMap *map, const void *pool, long long rows, int head_dim) {
+  auto fn = encode_tiled_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(pool), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK:
+      return "ok";
+    case PKV_EINVAL:
+      return "invalid argument";
+    case PKV_EUNSUPPORTED:
+      return "unsupported configuration";
+    case PKV_ECUDA:
+      return "CUDA error";
+    default:
+      return "unknown status";
+  }
+}
+
+size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
+                                  int partition_size) {
+  if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
+      partition_size < 0)
+    return 0;
+  const long long mp = parts_for(max_context_len, partition_size);
+  if (mp <= 1) return 0;
+  size_t off;
+  return workspace_layout(num_seqs, num_heads, head_dim, mp, &off);
+}
+
+int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
+                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                      int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                      int32_t *err, void *stream) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
+      partition_size < 0)
+    return PKV_EINVAL;
+  if (dtype < PKV_F32 || dtype > PKV_BF16) return PKV_EINVAL;
+  if (num_heads % num_kv_heads != 0) return PKV_EINVAL;
+  if (!isfinite(scale)) return PKV_EINVAL;
+  if (partition_size % 16 != 0) return PKV_EINVAL;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens) return PKV_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return PKV_EUNSUPPORTED;
+  if (num_seqs > 65535 || num_heads > 65535) return PKV_EUNSUPPORTED;
+
+  const uintptr_t al = dtype == PKV_F32 ? 4 : 16;
+  if (!aligned(out, al) || !aligned(q, al) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return PKV_EINVAL;
+
+  const long long mp = parts_for(max_context_len, partition_size);
+  if (mp > 0x7fffffffLL) return PKV_EUNSUPPORTED;
+  pkv::DecodeArgs a{};
+  a.out = out;
+  a.q = q;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.num_seqs = num_seqs;
+  a.num_heads = num_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.max_context_len = max_context_len;
+  a.max_parts = (int)mp;
+  if (partition_size > 0) {
+    a.part_tokens = partition_size;
+  } else {
+    const long long whole = round_up((size_t)(max_context_len > 0 ? max_context_len : 1), 16);
+    if (whole > 0x7fffffffLL) return PKV_EUNSUPPORTED;
+    a.part_tokens = (int)whole;
+  }
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.err = err;
+  if (mp > 1) {
+    size_t lse_off;
+    const size_t need = workspace_layout(num_seqs, num_heads, head_dim, mp, &lse_off);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return PKV_EINVAL;
+    a.ws_o = static_cast<float *>(workspace);
+    a.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + lse_off);
+  }
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == PKV_F32) {
+    e = pkv::launch_decode_simt_f32(a, st);
+  } else {
+    if (block_size % 16 != 0 || block_size > 256) return PKV_EUNSUPPORTED;
+    if (num_heads / num_kv_heads > 8) return PKV_EUNSUPPORTED;
+    if (num_kv_heads > 65535) return PKV_EUNSUPPORTED;
+    const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+    if (rows > 0x7fffffffLL - 64) return PKV_EUNSUPPORTED;
+    CUtensorMap tmK, tmV;
+    if (!make_pool_map(&tmK, k_pool, rows, head_dim) || !make_pool_map(&tmV, v_pool, rows, head_dim))
+      return PKV_ECUDA;
+    e = pkv::launch_decode_tc(a, dtype, tmK, tmV, st);
+  }
+  if (e != cudaSuccess) return PKV_ECUDA;
+  if (mp > 1) return cuda_status(pkv::launch_merge(a, dtype, st));
+  return PKV_OK;
+}
+
+int kv_cache_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,
+                    const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int dtype, int32_t *err, void *stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PKV_EINVAL;
+  if (dtype < PKV_F32 || dtype > PKV_BF16) return PKV_EINVAL;
+  if (num_tokens == 0) return PKV_OK;
+  if (!k_pool || !v_pool || !k_new || !v_new || !slot_mapping) return PKV_EINVAL;
+  const int es = dtype == PKV_F32 ? 4 : 2;
+  const long long row_bytes = (long long)head_dim * es;
+  if (row_bytes % 16 != 0 || row_bytes > 0x7fffffffLL) return PKV_EUNSUPPORTED;
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(slot_mapping, 8))
+    return PKV_EINVAL;
+  return cuda_status(pkv::launch_append(k_pool, v_pool, k_new, v_new, slot_mapping, num_tokens,
+                                        num_kv_heads, (int)row_bytes, block_size, num_blocks, err,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int kv_block_copy(void *k_pool, void *v_pool, const int32_t *src_dst, int num_pairs,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
+                  int32_t *err, void *stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+    return PKV_EINVAL;
+  if (dtype < PKV_F32 || dtype > PKV_BF16) return PKV_EINVAL;
+  if (num_pairs == 0) return PKV_OK;
+  if (!k_pool || !v_pool || !src_dst) return PKV_EINVAL;
+  const int es = dtype == PKV_F32 ? 4 : 2;
+  const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * es;
+  if (((long long)head_dim * es) % 16 != 0) return PKV_EUNSUPPORTED;
+  if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(src_dst, 4)) return PKV_EINVAL;
+  return cuda_status(pkv::launch_block_copy(k_pool, v_pool, src_dst, num_pairs, block_bytes,
+                                            num_blocks, err, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,225 @@
+// Paged decode attention for fp32 inputs, and the split-context merge.
+//
+// fp32 inputs keep fp32 arithmetic end to end: no tensor-core rounding of K,
+// V or P. One CTA (4 warps) attends one (sequence, query head, partition).
+// Each warp walks every 4th token: it looks up the token's physical block in
+// the block table, forms the score with a warp-wide dot product and updates a
+// running max / sum / output. That is the online walk of page "PagedAttention
+// Analysis" (ryotta.opik.net), section 3, one token at a time. The warps are
+// then combined in shared memory.
+//
+// The merge kernel combines the partitions of a split context. Partition p
+// contributes its normalised output o_p with weight 2^(lse_p - lse), where
+// lse_p is its base-2 log-sum-exp and lse = log2 sum_p 2^lse_p.
+#include "pkv_device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+constexpr int SIMT_WARPS = 4;
+
+template <int D>
+__global__ void __launch_bounds__(SIMT_WARPS * 32) decode_simt_f32_kernel(const DecodeArgs a) {
+  constexpr int E = D / 32;  // elements per lane
+  __shared__ float red_acc[SIMT_WARPS][D];
+  __shared__ float red_ml[SIMT_WARPS][2];
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int p = blockIdx.x;
+  const int hq = blockIdx.y;
+  const int s = blockIdx.z;
+  const int Hq = a.num_heads;
+  const int Hkv = a.num_kv_heads;
+  const int G = Hq / Hkv;
+  const int kvh = hq / G;
+  const int B = a.block_size;
+
+  const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, B,
+                              threadIdx.x == 0 ? a.err : nullptr);
+  float *out = static_cast<float *>(a.out);
+  const size_t row = (size_t)s * Hq + hq;
+  if (L <= 0) {
+    if (p == 0)
+      for (int d = threadIdx.x; d < D; d += SIMT_WARPS * 32) out[row * D + d] = 0.f;
+    return;
+  }
+  const int t_begin = p * a.part_tokens;
+  if (t_begin >= L) return;
+  const int t_end = min(L, t_begin + a.part_tokens);
+  const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
+
+  const float *qrow = static_cast<const float *>(a.q) + row * D;
+  float qv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) qv[e] = qrow[lane * E + e];
+
+  const float *kp = static_cast<const float *>(a.k_pool);
+  const float *vp = static_cast<const float *>(a.v_pool);
+  const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
+
+  float m = -INFINITY, l = 0.f, acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+
+  for (int t = t_begin + warp; t < t_end; t += SIMT_WARPS) {
+    const int phys = bt[t / B];
+    if (phys < 0 || phys >= a.num_blocks) {
+      if (lane == 0) report(a.err, PKV_DEV_BAD_BLOCK);
+      continue;
+    }
+    const size_t base = (((size_t)phys * Hkv + kvh) * B + (t % B)) * D + lane * E;
+    float dot = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kp[base + e], dot);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, off);
+    const float x = dot * a.scale_log2;
+    const float mn = fmaxf(m, x);
+    const float al = exp2f(m - mn);
+    const float pr = exp2f(x - mn);
+    l = l * al + pr;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = fmaf(pr, vp[base + e], acc[e] * al);
+    m = mn;
+  }
+
+#pragma unroll
+  for (int e = 0; e < E; ++e) red_acc[warp][lane * E + e] = acc[e];
+  if (lane == 0) {
+    red_ml[warp][0] = m;
+    red_ml[warp][1] = l;
+  }
+  __syncthreads();
+
+  for (int d = threadIdx.x; d < D; d += SIMT_WARPS * 32) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < SIMT_WARPS; ++w) M = fmaxf(M, red_ml[w][0]);
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < SIMT_WARPS; ++w) {
+        const float f = exp2f(red_ml[w][0] - M);
+        num += f * red_acc[w][d];
+        den += f * red_ml[w][1];
+      }
+    }
+    const float o = den > 0.f ? num / den : 0.f;
+    if (nparts == 1) {
+      out[row * D + d] = o;
+    } else {
+      a.ws_o[(row * a.max_parts + p) * D + d] = o;
+      if (d == 0) a.ws_lse[row * a.max_parts + p] = den > 0.f ? M + log2f(den) : -INFINITY;
+    }
+  }
+}
+
+constexpr int MERGE_THREADS = 256;
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float *scratch) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(FULL_MASK, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  v = scratch[0];
+  for (int w = 1; w < MERGE_THREADS / 32; ++w) v = is_max ? fmaxf(v, scratch[w]) : v + scratch[w];
+  return v;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const DecodeArgs a) {
+  constexpr int V = D / 4;               // float4 per row
+  constexpr int R = MERGE_THREADS / V;   // partition rows read concurrently
+  __shared__ float scratch[MERGE_THREADS / 32];
+  __shared__ float4 red[MERGE_THREADS];
+
+  const int hq = blockIdx.x;
+  const int s = blockIdx.y;
+  const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, a.block_size,
+                              nullptr);
+  const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
+  if (nparts <= 1) return;  // written directly by the decode kernel
+
+  const size_t row = (size_t)s * a.num_heads + hq;
+  const float *lse = a.ws_lse + row * a.max_parts;
+  const int tid = threadIdx.x;
+
+  float mx = -INFINITY;
+  for (int q = tid; q < nparts; q += MERGE_THREADS) mx = fmaxf(mx, lse[q]);
+  mx = block_reduce(mx, true, scratch);
+  float sum = 0.f;
+  if (mx != -INFINITY)
+    for (int q = tid; q < nparts; q += MERGE_THREADS) sum += exp2f(lse[q] - mx);
+  sum = block_reduce(sum, false, scratch);
+
+  const int r = tid / V, cv = tid - (tid / V) * V;
+  const float4 *po = reinterpret_cast<const float4 *>(a.ws_o + row * a.max_parts * D);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (mx != -INFINITY) {
+#pragma unroll 4
+    for (int q = r; q < nparts; q += R) {
+      const float w = exp2f(lse[q] - mx);
+      const float4 v = po[(size_t)q * V + cv];
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+  }
+  red[tid] = acc;
+  __syncthreads();
+  if (r == 0) {
+    float4 t = red[cv];
+    for (int rr = 1; rr < R; ++rr) {
+      const float4 u = red[rr * V + cv];
+      t.x += u.x;
+      t.y += u.y;
+      t.z += u.z;
+      t.w += u.w;
+    }
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    T *out = static_cast<T *>(a.out) + row * D + 4 * cv;
+    out[0] = from_float<T>(t.x * inv);
+    out[1] = from_float<T>(t.y * inv);
+    out[2] = from_float<T>(t.z * inv);
+    out[3] = from_float<T>(t.w * inv);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_merge_t(const DecodeArgs &a, cudaStream_t stream) {
+  dim3 grid(a.num_heads, a.num_seqs);
+  merge_kernel<T, D><<<grid, MERGE_THREADS, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream) {
+  dim3 grid(a.max_parts, a.num_heads, a.num_seqs);
+  if (a.head_dim == 64)
+    decode_simt_f32_kernel<64><<<grid, SIMT_WARPS * 32, 0, stream>>>(a);
+  else
+    decode_simt_f32_kernel<128><<<grid, SIMT_WARPS * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const DecodeArgs &a, int dtype, cudaStream_t stream) {
+  if (dtype == PKV_F32)
+    return a.head_dim == 64 ? launch_merge_t<float, 64>(a, stream)
+                            : launch_merge_t<float, 128>(a, stream);
+  if (dtype == PKV_F16)
+    return a.head_dim == 64 ? launch_merge_t<__half, 64>(a, stream)
+                            : launch_merge_t<__half, 128>(a, stream);
+  return a.head_dim == 64 ? launch_merge_t<__nv_bfloat16, 64>(a, stream)
+                          : launch_merge_t<__nv_bfloat16, 128>(a, stream);
+}
+
+}  // namespace pkv

@@ -1,0 +1,49 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+// Everything a decode launch needs, as plain values (kernel parameter block).
+struct DecodeArgs {
+  void *out;
+  const void *q;
+  const void *k_pool;
+  const void *v_pool;
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  float *ws_o;    // [S][Hq][max_parts][D] partition outputs (normalised), or null
+  float *ws_lse;  // [S][Hq][max_parts] partition log2-sum-exp, or null
+  int num_seqs;
+  int num_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks;      // block-table row length
+  int num_blocks;      // pool size in blocks
+  int max_context_len; // host upper bound on context_lens
+  int part_tokens;     // tokens per partition (multiple of 16)
+  int max_parts;       // partitions of the longest allowed context
+  float scale_log2;    // scale * log2(e): scores are kept in base-2 units
+  int32_t *err;        // nullable device error word
+};
+
+cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
+                             const CUtensorMap &tmV, cudaStream_t stream);
+cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeArgs &a, int dtype, cudaStream_t stream);
+
+cudaError_t launch_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,
+                          const int64_t *slots, int num_tokens, int num_kv_heads, int row_bytes,
+                          int block_size, int num_blocks, int32_t *err, cudaStream_t stream);
+cudaError_t launch_block_copy(void *k_pool, void *v_pool, const int32_t *pairs, int num_pairs,
+                              long long block_bytes, int num_blocks, int32_t *err,
+                              cudaStream_t stream);
+
+// Shared-memory bytes a decode_tc launch requests (for occupancy queries).
+size_t decode_tc_smem_bytes(int head_dim);
+
+}  // namespace pkv

@@ -1,0 +1,106 @@
+"""The C-ABI library on a host without a GPU: it builds, loads, exports every
+function ``include/pkv.h`` declares, and its synchronous argument checks
+return the documented status codes. Only calls rejected before any launch are
+made here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_387_b200 as pkv
+from paged_kv_cache_387_b200 import build as pkv_build
+
+HEADER_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([A-Za-z_]\w*)\s*\(", text, flags=re.M):
+            line = m.group(0)
+            if line.startswith(("typedef", "#", "enum", "return")):
+                continue
+            names.append(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pkv_build.build()
+    return pkv.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(pkv.EXPORTS) <= set(names), names
+    raw = ctypes.CDLL(pkv.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings(lib):
+    assert lib.pkv_status_string(0) == b"ok"
+    assert lib.pkv_status_string(-1) == b"invalid argument"
+    assert lib.pkv_status_string(-2) == b"unsupported configuration"
+    assert lib.pkv_status_string(-3) == b"CUDA error"
+
+
+def test_workspace_arithmetic(lib):
+    f = lib.pkv_decode_workspace_bytes
+    assert f(8, 32, 128, 512, 512) == 0          # one partition: no workspace
+    assert f(8, 32, 128, 100, 0) == 0            # unsplit
+    # 8 seqs x 32 heads x 256 partitions: fp32 outputs [..][128] + one lse each
+    assert f(8, 32, 128, 131072, 512) == 8 * 32 * 256 * 128 * 4 + 8 * 32 * 256 * 4
+    # 33 tokens in 16-token partitions = 3 partitions; regions are 256-byte aligned
+    assert f(1, 1, 64, 33, 16) == 3 * 64 * 4 + 256
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below is rejected first
+
+
+def decode(lib, **kw):
+    args = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, cl=FAKE, S=2, Hq=8, Hkv=2, D=128,
+                B=16, MB=4, P=10, L=64, scale=0.088, dtype=2, part=512, ws=None, wsb=0,
+                err=None, stream=None)
+    args.update(kw)
+    return lib.paged_attn_decode(*args.values())
+
+
+def test_decode_argument_checks(lib):
+    assert decode(lib, out=None) == pkv.PKV_EINVAL
+    assert decode(lib, Hq=6, Hkv=4) == pkv.PKV_EINVAL
+    assert decode(lib, part=24) == pkv.PKV_EINVAL
+    assert decode(lib, dtype=7) == pkv.PKV_EINVAL
+    assert decode(lib, scale=float("nan")) == pkv.PKV_EINVAL
+    assert decode(lib, L=2048, ws=None, wsb=0) == pkv.PKV_EINVAL     # workspace needed
+    assert decode(lib, D=96) == pkv.PKV_EUNSUPPORTED
+    assert decode(lib, B=8) == pkv.PKV_EUNSUPPORTED                   # 16-bit needs B % 16 == 0
+    assert decode(lib, Hq=32, Hkv=2) == pkv.PKV_EUNSUPPORTED          # group of 16 > 8
+    assert decode(lib, q=ctypes.c_void_p(0x10008)) == pkv.PKV_EINVAL  # misaligned
+    assert decode(lib, S=0) == pkv.PKV_OK                             # nothing to do
+
+
+def test_append_and_copy_argument_checks(lib):
+    ap = lib.kv_cache_append
+    assert ap(FAKE, FAKE, FAKE, FAKE, None, 4, 2, 128, 16, 10, 1, None, None) == pkv.PKV_EINVAL
+    assert ap(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 4, 16, 10, 1, None, None) == pkv.PKV_EUNSUPPORTED
+    assert ap(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, 128, 16, 10, 1, None, None) == pkv.PKV_OK
+    cp = lib.kv_block_copy
+    assert cp(FAKE, None, FAKE, 3, 2, 128, 16, 10, 1, None, None) == pkv.PKV_EINVAL
+    assert cp(FAKE, FAKE, FAKE, -1, 2, 128, 16, 10, 1, None, None) == pkv.PKV_EINVAL
+    assert cp(FAKE, FAKE, None, 0, 2, 128, 16, 10, 1, None, None) == pkv.PKV_OK
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
