@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b_gqa_b256")
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="keep only the first sequences of the workload (small profiling cases)")
     ap.add_argument("--soak-seconds", type=float, default=2.0,
                     help="back-to-back steps before the timed region (clock sampling, warm clocks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -224,7 +226,8 @@ def run_reference(args, rank, world):
     from pkv_inputs import make_case
     oracle.build()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    case = make_case(args.workload, device=dev, with_append=True).to("cpu")
+    case = make_case(args.workload, device=dev, with_append=True,
+                     num_seqs=args.num_seqs).to("cpu")
     budget = 150.0  # seconds for warmup + steps
     per_step = min(2.0, budget / max(1, args.steps + args.warmup))
     nseq = size_oracle_sample(case, per_step)
@@ -288,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    case = make_case(args.workload, device=dev, with_append=True)
+    case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs)
     stream = torch.cuda.current_stream(dev)
 
     S, Hq, D = case.num_seqs, case.num_heads, case.head_dim
@@ -398,7 +401,8 @@ def run_ours(args, rank, world, local_rank):
 
     contiguous = None
     if args.contiguous:
-        ccase = make_case(args.workload, device=dev, with_append=False, placement="identity")
+        ccase = make_case(args.workload, device=dev, with_append=False, placement="identity",
+                          num_seqs=args.num_seqs)
         cout = torch.empty_like(ccase.q)
         for _ in range(3):
             decode(ccase, cout)

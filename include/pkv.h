@@ -66,9 +66,12 @@ enum {
 };
 
 /*
- * Bytes of device workspace paged_attn_decode needs for these sizes. The
- * answer is 0 when no sequence needs more than one partition. This function
- * is pure arithmetic: it does not touch the GPU.
+ * Bytes of device workspace paged_attn_decode needs for these sizes: a few
+ * scheduling words and the work list (one 4-byte entry per possible
+ * (sequence, partition) pair), plus, when a context can span several
+ * partitions, one fp32 output row and one fp32 log-sum-exp per (sequence,
+ * query head, partition). Always > 0 for num_seqs > 0. This function is pure
+ * arithmetic: it does not touch the GPU.
  */
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_context_len, int partition_size);
@@ -108,8 +111,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
  * partition_size tokens per partition. 0 means no split (one partition of
  *                the whole context). Otherwise a positive multiple of 16.
  * workspace      device scratch of at least pkv_decode_workspace_bytes(...)
- *                bytes, 16-byte aligned. It may be NULL when that size is 0.
- *                Its contents on entry do not matter.
+ *                bytes, 256-byte aligned. Its contents on entry do not
+ *                matter. Calls that overlap in time must not share it.
  * err            nullable device int32 error word (see above).
  *
  * Supported: head_dim in {64, 128}; f32 with any block_size >= 1; f16/bf16

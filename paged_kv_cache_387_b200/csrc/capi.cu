@@ -22,16 +22,6 @@ long long parts_for(int max_context_len, int partition_size) {
   return (L + partition_size - 1) / partition_size;
 }
 
-// Workspace = [S][Hq][max_parts][D] float partials, then [S][Hq][max_parts]
-// float log2-sum-exp values, each region 256-byte aligned.
-size_t workspace_layout(long long S, long long Hq, long long D, long long max_parts,
-                        size_t *lse_offset) {
-  const size_t o_bytes = round_up((size_t)(S * Hq * max_parts * D) * sizeof(float), 256);
-  const size_t l_bytes = round_up((size_t)(S * Hq * max_parts) * sizeof(float), 256);
-  *lse_offset = o_bytes;
-  return o_bytes + l_bytes;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -66,6 +56,38 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
 
 }  // namespace
 
+namespace pkv {
+
+WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long long max_parts) {
+  WorkspaceLayout w{};
+  size_t off = 0;
+  w.sched_off = off;
+  off += 256;
+  w.work_off = off;
+  off += round_up((size_t)(S * max_parts) * sizeof(uint32_t), 256);
+  if (max_parts > 1) {
+    const long long chunks = (max_parts + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK;
+    w.cnt_off = off;  // Hq >= Hkv bounds the (sequence, KV head) counters
+    off += round_up((size_t)(S * Hq * chunks) * sizeof(int32_t), 256);
+    w.cnt2_off = off;
+    off += round_up((size_t)(S * Hq) * sizeof(int32_t), 256);
+    w.o_off = off;
+    off += round_up((size_t)(S * Hq * max_parts * D) * sizeof(float), 256);
+    w.lse_off = off;
+    off += round_up((size_t)(S * Hq * max_parts) * sizeof(float), 256);
+    if (chunks > 1) {
+      w.o2_off = off;
+      off += round_up((size_t)(S * Hq * chunks * D) * sizeof(float), 256);
+      w.lse2_off = off;
+      off += round_up((size_t)(S * Hq * chunks) * sizeof(float), 256);
+    }
+  }
+  w.total = off;
+  return w;
+}
+
+}  // namespace pkv
+
 extern "C" {
 
 const char *pkv_status_string(int status) {
@@ -89,9 +111,7 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int
       partition_size < 0)
     return 0;
   const long long mp = parts_for(max_context_len, partition_size);
-  if (mp <= 1) return 0;
-  size_t off;
-  return workspace_layout(num_seqs, num_heads, head_dim, mp, &off);
+  return pkv::workspace_layout(num_seqs, num_heads, head_dim, mp).total;
 }
 
 int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
@@ -118,8 +138,15 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
       !aligned(block_tables, 4) || !aligned(context_lens, 4))
     return PKV_EINVAL;
 
+  long long rows = 0;  // pool rows of the TMA view (16-bit path)
+  if (dtype != PKV_F32) {
+    if (block_size % 16 != 0 || block_size > 256) return PKV_EUNSUPPORTED;
+    if (num_heads / num_kv_heads > 8) return PKV_EUNSUPPORTED;
+    rows = (long long)num_blocks * num_kv_heads * block_size;
+    if (rows > 0x7fffffffLL - 64) return PKV_EUNSUPPORTED;
+  }
   const long long mp = parts_for(max_context_len, partition_size);
-  if (mp > 0x7fffffffLL) return PKV_EUNSUPPORTED;
+  if (mp > 65535) return PKV_EUNSUPPORTED;  // work-list entries pack the partition in 16 bits
   pkv::DecodeArgs a{};
   a.out = out;
   a.q = q;
@@ -145,12 +172,21 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
   }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.err = err;
+  const pkv::WorkspaceLayout wl = pkv::workspace_layout(num_seqs, num_heads, head_dim, mp);
+  if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 256)) return PKV_EINVAL;
+  char *ws = static_cast<char *>(workspace);
+  a.sched = reinterpret_cast<int32_t *>(ws + wl.sched_off);
+  a.work = reinterpret_cast<uint32_t *>(ws + wl.work_off);
+  a.max_chunks = (int)((mp + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK);
   if (mp > 1) {
-    size_t lse_off;
-    const size_t need = workspace_layout(num_seqs, num_heads, head_dim, mp, &lse_off);
-    if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return PKV_EINVAL;
-    a.ws_o = static_cast<float *>(workspace);
-    a.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + lse_off);
+    a.merge_cnt = reinterpret_cast<int32_t *>(ws + wl.cnt_off);
+    a.merge_cnt2 = reinterpret_cast<int32_t *>(ws + wl.cnt2_off);
+    if (a.max_chunks > 1) {
+      a.ws2_o = reinterpret_cast<float *>(ws + wl.o2_off);
+      a.ws2_lse = reinterpret_cast<float *>(ws + wl.lse2_off);
+    }
+    a.ws_o = reinterpret_cast<float *>(ws + wl.o_off);
+    a.ws_lse = reinterpret_cast<float *>(ws + wl.lse_off);
   }
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -158,15 +194,11 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
   if (dtype == PKV_F32) {
     e = pkv::launch_decode_simt_f32(a, st);
   } else {
-    if (block_size % 16 != 0 || block_size > 256) return PKV_EUNSUPPORTED;
-    if (num_heads / num_kv_heads > 8) return PKV_EUNSUPPORTED;
-    if (num_kv_heads > 65535) return PKV_EUNSUPPORTED;
-    const long long rows = (long long)num_blocks * num_kv_heads * block_size;
-    if (rows > 0x7fffffffLL - 64) return PKV_EUNSUPPORTED;
     CUtensorMap tmK, tmV;
     if (!make_pool_map(&tmK, k_pool, rows, head_dim) || !make_pool_map(&tmV, v_pool, rows, head_dim))
       return PKV_ECUDA;
-    e = pkv::launch_decode_tc(a, dtype, tmK, tmV, st);
+    // plan + decode; the partition merge is fused into the decode kernel
+    return cuda_status(pkv::launch_decode_tc(a, dtype, tmK, tmV, st));
   }
   if (e != cudaSuccess) return PKV_ECUDA;
   if (mp > 1) return cuda_status(pkv::launch_merge(a, dtype, st));

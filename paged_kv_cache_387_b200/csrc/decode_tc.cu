@@ -1,8 +1,8 @@
 // Paged decode attention for fp16 / bf16 on sm_100a.
 //
-// One CTA attends one (sequence, KV head, partition). It serves all
-// G = Hq/Hkv query heads of the KV head's group at once, so each K/V byte
-// is read from HBM once per group.
+// Work is one (sequence, partition, KV head) item. The whole group of
+// G = Hq/Hkv query heads that share the KV head is attended at once, so each
+// K/V byte is read from HBM once per group.
 //
 // The block-by-block online softmax is the walk over the block table in page
 // "PagedAttention Analysis" (ryotta.opik.net), section 3: look up each logical
@@ -11,352 +11,848 @@
 // the causal sum of page "PagedAttention" (newikis), section "Mathematical
 // formulation".
 //
-// Data movement
-//   The unit of work is a 16-token tile of one KV head: 16 rows of head_dim
-//   elements, a slice of one physical block (block_size is a multiple of 16).
-//   Each warp owns a 3-stage ring in shared memory. Lane 0 fetches a tile's K
-//   and V with 2D TMA loads of 64-element-wide boxes under the 128-byte
-//   swizzle and completes them on an mbarrier. A warp walks tiles w, w+4,
-//   w+8, ... of the partition. No load uses cluster multicast.
+// Scheduling
+//   A one-CTA plan kernel turns context_lens into a compact work list of
+//   (sequence, partition) pairs: full partitions first, then the shorter last
+//   partitions. It also resets the dispatch and merge counters. The decode
+//   kernel is persistent, two CTAs per SM, and pulls items (pair x KV head)
+//   from an atomic counter until the list is exhausted. It is launched as a
+//   programmatic dependent of the plan, so its set-up overlaps the plan.
 //
-// Math (per tile, per warp), fp32 accumulation:
-//   S^T[16 tok][8 heads] = K_tile[16][D] . Q^T[D][8]  mma.sync m16n8k16. K is
-//     the A operand, read straight from the swizzled tile. The D axis is
-//     visited in a lane-dependent order that Q's fragments follow too, which
-//     keeps every shared load a conflict-free 16-byte access. Q (G <= 8 heads,
-//     zero-padded to 8) stays in registers for the whole tile loop.
-//   online softmax in base 2 on the accumulator fragment. Masked tokens get
-//     -inf, and the V rows of masked tokens are zeroed in shared memory before
-//     they reach the tensor core.
+// Warp roles
+//   Warp 4 is the scheduler. It resolves items ahead of use (work-list
+//   entry, context length, the physical block id of every 16-token tile) and
+//   posts them as descriptors into a small ring, with the group's q rows
+//   fetched by one bulk copy. It also keeps the partition count. When the
+//   consumers finish an item of a split context, the scheduler publishes it
+//   (a device-scope fence and a fetch-and-add on the (sequence, KV head)
+//   counter). The CTA that completes the last partition receives a merge
+//   task in its descriptor stream. No CTA ever waits for another.
+//   Warps 0-3 are consumers. Each owns a ring of stages in shared memory and
+//   takes tiles w, w+4, w+8, ... of every item. Its lane 0 fills the ring
+//   with TMA: per tile, 2D loads of K and V (64-element boxes, 128-byte
+//   swizzle) completing on the stage's mbarrier. The fill runs ahead of the
+//   warp's math across item boundaries. No load uses cluster multicast.
+//
+// Math (per tile, per consumer warp), fp32 accumulation:
+//   S^T[16 tok][8] = K_tile[16][D] . Q^T[D][8]  mma.sync m16n8k16. K is the A
+//     operand, read straight from the swizzled tile. The D axis is visited in
+//     a lane-dependent order that Q's fragments follow too, which keeps every
+//     shared load a conflict-free 16-byte access. Q (the group's heads,
+//     zero-padded to 8) sits in registers for the whole item.
+//   online softmax in base 2 on the accumulator fragment. The running max
+//     moves only when a tile's max exceeds it by more than 2^8, which keeps
+//     rescaling rare. Masked tokens get -inf, and their V rows are zeroed in
+//     shared memory before they reach the tensor core.
 //   O^T[D][8] += V^T[D][16] . P^T[16][8]  V^T via ldmatrix.trans; P^T from the
 //     score fragment via movmatrix.trans (P rounded to the input type).
-// At the end the four warps' (max, sum, output) are combined in shared
-// memory. The result is written to `out` when the sequence has one partition,
-// and otherwise to the workspace as (normalised o_p, log2-sum-exp) for the
-// merge kernel.
+// At the end of an item the consumer warps' (max, sum, output) are combined in
+// shared memory. The result goes to `out` when the sequence has one
+// partition, and otherwise to the workspace as (normalised o_p,
+// log2-sum-exp). Every wait is bounded: one that gives up sets an error
+// status and a CTA-wide stop flag, and the kernel winds down.
 #include "pkv_device.cuh"
 #include "pkv_internal.h"
 
 namespace pkv {
 namespace {
 
-constexpr int TILE = 16;                   // tokens per tile (mma M for QK, K for PV)
-constexpr int NWARPS = 4;                  // warps per CTA
-constexpr int NSTAGE = 3;                  // ring depth per warp
-constexpr int BOX_COLS = 64;               // elements per TMA box row (128 bytes)
-constexpr int HALF_BYTES = TILE * 128;     // one box: 16 rows x 128 bytes
+constexpr int TILE = 16;                 // tokens per tile (mma M for QK, K for PV)
+constexpr int NCW = 4;                   // consumer warps
+constexpr int THREADS = (NCW + 1) * 32;  // + one scheduler warp
+constexpr int NSLOT = 3;                 // item descriptors in flight
+constexpr int DESC_TILES = 64;           // tile block ids carried by a descriptor
+constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
+constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
+constexpr int PLAN_THREADS = 1024;
+constexpr float RESCALE_SLACK = 8.f;     // lazy max: rescale only past 2^8 growth
 
-template <int D>
-struct TcShape {
-  static constexpr int HALVES = D / BOX_COLS;
-  static constexpr int KT_BYTES = HALVES * HALF_BYTES;     // one K (or V) tile
-  static constexpr int STAGE_BYTES = 2 * KT_BYTES;         // K + V
-  static constexpr int RING_BYTES = NWARPS * NSTAGE * STAGE_BYTES;
-  static constexpr int BAR_BYTES = NWARPS * NSTAGE * 8;
-  static constexpr int SMEM_BYTES = RING_BYTES + BAR_BYTES + 1024;  // + alignment slack
-  static constexpr int ACC_STRIDE = D + 4;  // padded row of the combine area (floats)
-  static_assert(8 * ACC_STRIDE * 4 + 64 <= NSTAGE * STAGE_BYTES, "combine area must fit");
+// Descriptor kinds (in ItemDesc::kind).
+constexpr int KIND_WORK = 0;         // attend one (sequence, partition, KV head)
+constexpr int KIND_MERGE_CHUNK = 1;  // merge partitions of chunk p into a chunk result
+constexpr int KIND_MERGE_FINAL = 2;  // merge partitions (one chunk) or chunk results into out
+constexpr int KIND_NOP = 3;          // keeps the ring turning while the last items finish
+constexpr int KIND_END = 4;          // no more descriptors
+constexpr int PLAN_BUCKETS = 64;     // size classes for ordering the short last partitions
+
+// One entry of the scheduler -> consumer descriptor ring.
+struct ItemDesc {
+  int kind, s, p, h, L, n_tiles, nparts, pad;
+  int ids[DESC_TILES];  // physical block of tile t (tiles beyond: read from the table)
 };
 
-template <typename T, int D>
-__global__ void __launch_bounds__(NWARPS * 32)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
-  using Shape = TcShape<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t smem0 = (raw_addr + 1023u) & ~1023u;  // 128B swizzle wants 1024B alignment
-  uint8_t *const smem_gen = smem_raw + (smem0 - raw_addr);
+// Shared-memory plan of one CTA (offsets from the 1024-aligned base). NH is
+// the number of head rows an instantiation carries (4 or 8 >= G).
+template <int D, int NH>
+struct TcShape {
+  static constexpr int HALVES = D / BOX_COLS;
+  static constexpr int KT_BYTES = HALVES * HALF_BYTES;   // one K (or V) tile
+  static constexpr int STAGE_BYTES = 2 * KT_BYTES;       // K + V
+  static constexpr int ACC_STRIDE = D + 4;               // padded combine row (floats)
+  static constexpr int CW_FLOATS = NH * ACC_STRIDE + 2 * NH;  // acc[NH][D+4], m[NH], l[NH]
+  static constexpr int COMBINE_BYTES = (NCW * CW_FLOATS + NH * (NCW + 1)) * 4;  // + scales
+  static constexpr int QBUF_BYTES = NH * D * 2;
+  static constexpr int FIXED = COMBINE_BYTES + NSLOT * QBUF_BYTES +
+                               NSLOT * (int)sizeof(ItemDesc) + 64 * 8 + 1024 + 64;
+  // As many stages as fit two CTAs per SM (about 110 KB each), at most 6.
+  static constexpr int NSTAGE_FIT = (110 * 1024 - FIXED) / (NCW * STAGE_BYTES);
+  static constexpr int NSTAGE = NSTAGE_FIT > 6 ? 6 : NSTAGE_FIT;
+  static_assert(NSTAGE >= 2, "ring too shallow");
+  static constexpr int RING_BYTES = NCW * NSTAGE * STAGE_BYTES;
+  static constexpr int COMBINE_OFF = RING_BYTES;
+  static constexpr int QBUF_OFF = COMBINE_OFF + ((COMBINE_BYTES + 15) & ~15);
+  static constexpr int DESC_OFF = QBUF_OFF + NSLOT * QBUF_BYTES;
+  static constexpr int BAR_OFF = DESC_OFF + NSLOT * (int)sizeof(ItemDesc);
+  static constexpr int NBARS = NCW * NSTAGE + 2 * NSLOT;
+  static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 1024;  // + alignment slack
+  static_assert(QBUF_OFF % 16 == 0 && DESC_OFF % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
+};
 
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int g = lane >> 2;  // mma group id (row of A / column of B)
-  const int c = lane & 3;   // thread in group
-  const int p = blockIdx.x;
-  const int h = blockIdx.y;
-  const int s = blockIdx.z;
-  const int Hq = a.num_heads;
-  const int G = Hq / a.num_kv_heads;
-  const int B = a.block_size;
+__device__ __forceinline__ uint32_t pack_pair(int s, int p) {
+  return (static_cast<uint32_t>(s) << 16) | static_cast<uint32_t>(p);
+}
 
-  const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, B,
-                              threadIdx.x == 0 ? a.err : nullptr);
-  T *const out = static_cast<T *>(a.out);
-  if (L <= 0) {
-    if (p == 0)
-      for (int idx = threadIdx.x; idx < G * D; idx += NWARPS * 32)
-        out[((size_t)s * Hq + h * G) * D + idx] = from_float<T>(0.f);
-    return;
+// Build the work list: every sequence's full partitions first (all the same
+// size), then the shorter last partitions ordered by size, largest first
+// (a counting sort over PLAN_BUCKETS size classes). Handing out the largest
+// items first and the smallest last keeps the CTAs' finishing times close. A
+// sequence of length 0 gets one entry, so its output is still written. The
+// merge counters are reset here too.
+__global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
+  __shared__ int wsum[PLAN_THREADS / 32];
+  __shared__ int hist[PLAN_BUCKETS];
+  pdl_launch_dependents();  // the decode grid may launch; it waits for this grid to finish
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int S = a.num_seqs, P = a.part_tokens;
+  if (a.merge_cnt) {
+    const int n1 = S * a.num_kv_heads * a.max_chunks;
+    for (int i = tid; i < n1; i += PLAN_THREADS) a.merge_cnt[i] = 0;
+    for (int i = tid; i < S * a.num_kv_heads; i += PLAN_THREADS) a.merge_cnt2[i] = 0;
   }
-  const int t_begin = p * a.part_tokens;
-  if (t_begin >= L) return;
-  const int t_end = min(L, t_begin + a.part_tokens);
-  const int n_tiles = (t_end - t_begin + TILE - 1) / TILE;
-  const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
-  const int nt_w = warp < n_tiles ? (n_tiles - warp + NWARPS - 1) / NWARPS : 0;
-
-  const uint32_t ring = smem0 + warp * NSTAGE * Shape::STAGE_BYTES;
-  const uint32_t bar0 = smem0 + Shape::RING_BYTES + warp * NSTAGE * 8;
-  if (lane == 0) {
-    for (int st = 0; st < NSTAGE; ++st) mbar_init(bar0 + 8 * st, 1);
-    fence_mbar_init();
-  }
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-  }
-  __syncwarp();
-
-  // Q^T as the B operand: lane (g, c) holds head g's elements
-  // 8*Lc .. 8*Lc+7 for logical chunk Lc(c, j) = (j/2)*8 + 2c + (j%2).
-  uint4 qf[D / 32];
-  {
-    const bool head_ok = g < G;
-    const T *qrow = static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G + (head_ok ? g : 0)) * D;
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      const int Lc = (j >> 1) * 8 + 2 * c + (j & 1);
-      qf[j] = head_ok ? *reinterpret_cast<const uint4 *>(qrow + Lc * 8) : make_uint4(0, 0, 0, 0);
-    }
-  }
-
-  // Physical block ids of this warp's tiles, 32 at a time (lane j <-> tile win_base + j).
-  const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
-  auto tile_tok0 = [&](int i) { return t_begin + (warp + i * NWARPS) * TILE; };
-  int win_base = 0;
-  int win_id = lane < nt_w ? bt[tile_tok0(lane) / B] : -1;
-  const int total_rows = a.num_blocks * a.num_kv_heads * B;
-  uint32_t bad_mask = 0;  // bit st: the tile in stage st had an invalid block id
-
-  // Warp-wide: fetch tile i into stage i % NSTAGE.
-  auto issue = [&](int i) {
-    if (i - win_base >= 32) {
-      win_base += 32;
-      const int k = win_base + lane;
-      win_id = k < nt_w ? bt[tile_tok0(k) / B] : -1;
-    }
-    const int phys = __shfl_sync(FULL_MASK, win_id, i - win_base);
-    const int st = i % NSTAGE;
-    const bool bad = phys < 0 || phys >= a.num_blocks;
-    bad_mask = bad ? (bad_mask | (1u << st)) : (bad_mask & ~(1u << st));
-    if (lane == 0) {
-      int y;
-      if (bad) {
-        report(a.err, PKV_DEV_BAD_BLOCK);
-        y = total_rows;  // wholly out of bounds: TMA fills zeros
-      } else {
-        y = (phys * a.num_kv_heads + h) * B + (tile_tok0(i) % B);
-      }
-      const uint32_t bar = bar0 + 8 * st;
-      const uint32_t kdst = ring + st * Shape::STAGE_BYTES;
-      const uint32_t vdst = kdst + Shape::KT_BYTES;
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, Shape::STAGE_BYTES);
-#pragma unroll
-      for (int hh = 0; hh < Shape::HALVES; ++hh) {
-        tma_load_2d(kdst + hh * HALF_BYTES, &tmK, hh * BOX_COLS, y, bar);
-        tma_load_2d(vdst + hh * HALF_BYTES, &tmV, hh * BOX_COLS, y, bar);
-      }
-    }
+  if (tid < PLAN_BUCKETS) hist[tid] = 0;
+  __syncthreads();
+  const int chunk = (S + PLAN_THREADS - 1) / PLAN_THREADS;
+  const int s0 = min(S, tid * chunk), s1 = min(S, s0 + chunk);
+  const int max_tiles = max(1, P / 16);
+  // size class of a last partition of `rem` tokens: bigger -> smaller bucket
+  auto bucket = [&](int rem) {
+    const int tiles = (rem + 15) / 16;
+    return (PLAN_BUCKETS - 1) - min(PLAN_BUCKETS - 1, tiles * (PLAN_BUCKETS - 1) / max_tiles);
   };
 
-  float acc[D / 16][4];
-#pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2c, 2c+1 (base-2 units)
-  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
-  const float sl2 = a.scale_log2;
-
-  const int pre = nt_w < NSTAGE ? nt_w : NSTAGE;
-  for (int i = 0; i < pre; ++i) issue(i);
-
-  // ldmatrix.trans row addresses for V: lane feeds row (lane & 7) of matrix lane >> 3.
-  const int mi = lane >> 3;
-  const int vr = (lane & 7) + ((mi >> 1) << 3);  // token row inside the tile
-
-  // A wait that gives up (never expected: a TMA load completes in microseconds)
-  // ends this warp's loop with an error status instead of spinning on. CTAs
-  // that start after such a report skip their waits too, so a failure cannot
-  // turn into a long stall.
-  bool aborted = a.err != nullptr &&
-                 *reinterpret_cast<volatile const int32_t *>(a.err) == PKV_DEV_WAIT_TIMEOUT;
-
-  for (int i = 0; i < nt_w && !aborted; ++i) {
-    const int st = i % NSTAGE;
-    const uint32_t bar = bar0 + 8 * st;
-    const uint32_t parity = (i / NSTAGE) & 1;
-    const bool ok = __all_sync(FULL_MASK, mbar_wait_bounded(bar, parity));
-    if (!ok) {
-      if (lane == 0) report(a.err, PKV_DEV_WAIT_TIMEOUT);
-      aborted = true;
-      break;
-    }
-    const uint32_t ks = ring + st * Shape::STAGE_BYTES;
-    const uint32_t vs = ks + Shape::KT_BYTES;
-    const int tok0 = tile_tok0(i);
-    const int valid = min(TILE, L - tok0);
-    const bool bad = (bad_mask >> st) & 1u;
-
-    if (valid < TILE && !bad) {
-      // Tokens past the context length: their V rows may hold anything
-      // (NaN included); zero them so P*V stays finite.
-      const int nchunks = (TILE - valid) * 8 * Shape::HALVES;
-      for (int e = lane; e < nchunks; e += 32) {
-        const int r = valid + e / (8 * Shape::HALVES);
-        const int rem = e % (8 * Shape::HALVES);
-        sts128_zero(vs + (rem >> 3) * HALF_BYTES + r * 128 + (rem & 7) * 16);
-      }
-      __syncwarp();
-    }
-
-    // ---- scores: S^T = K . Q^T ----
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      const int Lc = (j >> 1) * 8 + 2 * c + (j & 1);
-      const uint32_t rowg = ks + (Lc >> 3) * HALF_BYTES + g * 128 + (((Lc & 7) ^ g) << 4);
-      const uint4 ka = lds128(rowg);             // token g
-      const uint4 kb = lds128(rowg + 8 * 128);   // token g + 8 (same swizzle phase)
-      mma16816<T>(sc, ka.x, kb.x, ka.y, kb.y, qf[j].x, qf[j].y);
-      mma16816<T>(sc, ka.z, kb.z, ka.w, kb.w, qf[j].z, qf[j].w);
-    }
-
-    // ---- online softmax (heads 2c, 2c+1; tokens g, g+8) ----
-    const bool ok0 = !bad && g < valid;
-    const bool ok1 = !bad && g + 8 < valid;
-    const float x0 = ok0 ? sc[0] * sl2 : -INFINITY;
-    const float x1 = ok0 ? sc[1] * sl2 : -INFINITY;
-    const float x2 = ok1 ? sc[2] * sl2 : -INFINITY;
-    const float x3 = ok1 ? sc[3] * sl2 : -INFINITY;
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
-    const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float al0 = ex2_approx(m0 - mu0), al1 = ex2_approx(m1 - mu1);
-    const float p0 = ex2_approx(x0 - mu0), p1 = ex2_approx(x1 - mu1);
-    const float p2 = ex2_approx(x2 - mu0), p3 = ex2_approx(x3 - mu1);
-    l0 = l0 * al0 + (p0 + p2);
-    l1 = l1 * al1 + (p1 + p3);
-    m0 = mn0;
-    m1 = mn1;
-#pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      acc[mt][0] *= al0;
-      acc[mt][1] *= al1;
-      acc[mt][2] *= al0;
-      acc[mt][3] *= al1;
-    }
-
-    // P^T as the B operand: transpose the (token, head) fragment pairs.
-    const uint32_t pb0 = movmatrix_trans(pack2<T>(p0, p1));  // tokens 0..7
-    const uint32_t pb1 = movmatrix_trans(pack2<T>(p2, p3));  // tokens 8..15
-
-    // ---- O^T += V^T . P^T ----
-    const uint32_t vrow = vs + vr * 128;
-#pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      const int chunk = 2 * mt + (mi & 1);
-      const uint32_t addr = vrow + (chunk >> 3) * HALF_BYTES + (((chunk & 7) ^ (vr & 7)) << 4);
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4_trans(addr, r0, r1, r2, r3);
-      mma16816<T>(acc[mt], r0, r1, r2, r3, pb0, pb1);
-    }
-    __syncwarp();
-    if (i + NSTAGE < nt_w) issue(i + NSTAGE);
+  int nf = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
+                                a.block_size, nullptr);
+    nf += L / P;
+    const int rem = L % P;
+    if (rem != 0 || L == 0) atomicAdd(&hist[bucket(rem)], 1);
   }
-
-  // Full per-warp sums: add the 8 lanes that share a head pair.
+  // block-wide exclusive scan of the full-partition counts
+  int f = nf;
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l0 += __shfl_xor_sync(FULL_MASK, l0, off);
-    l1 += __shfl_xor_sync(FULL_MASK, l1, off);
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(FULL_MASK, f, off);
+    if (lane >= off) f += y;
   }
-
-  // ---- combine the warps (their rings are idle now: every issued tile was consumed) ----
+  if (lane == 31) wsum[warp] = f;
   __syncthreads();
-  constexpr int AS = Shape::ACC_STRIDE;
-  {
-    float *cw = reinterpret_cast<float *>(smem_gen + warp * NSTAGE * Shape::STAGE_BYTES);
+  if (warp == 0) {
+    int v = wsum[lane];
 #pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      cw[(2 * c) * AS + 16 * mt + g] = acc[mt][0];
-      cw[(2 * c + 1) * AS + 16 * mt + g] = acc[mt][1];
-      cw[(2 * c) * AS + 16 * mt + g + 8] = acc[mt][2];
-      cw[(2 * c + 1) * AS + 16 * mt + g + 8] = acc[mt][3];
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(FULL_MASK, v, off);
+      if (lane >= off) v += y;
     }
-    if (g == 0) {
-      cw[8 * AS + 2 * c] = m0;
-      cw[8 * AS + 2 * c + 1] = m1;
-      cw[8 * AS + 8 + 2 * c] = l0;
-      cw[8 * AS + 8 + 2 * c + 1] = l1;
+    wsum[lane] = v;  // inclusive prefix over warps
+  }
+  __syncthreads();
+  const int base_f = (warp ? wsum[warp - 1] : 0) + f - nf;
+  const int total_f = wsum[PLAN_THREADS / 32 - 1];
+  // bucket offsets (exclusive scan of hist, after the full partitions)
+  if (warp == 0) {
+    const int h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
+    int v = h0 + h1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(FULL_MASK, v, off);
+      if (lane >= off) v += y;
+    }
+    const int excl = v - h0 - h1;
+    hist[2 * lane] = total_f + excl;
+    hist[2 * lane + 1] = total_f + excl + h0;
+    if (lane == 31 && tid == 31) {
+      a.sched[0] = 0;
+      a.sched[1] = total_f + v;
     }
   }
   __syncthreads();
 
-  const bool single = nparts == 1;
-  for (int idx = threadIdx.x; idx < G * D; idx += NWARPS * 32) {
-    const int n = idx / D;
-    const int d = idx - n * D;
+  int of = base_f;
+  for (int s = s0; s < s1; ++s) {
+    const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
+                                a.block_size, nullptr);
+    const int full = L / P;
+    for (int q = 0; q < full; ++q) a.work[of++] = pack_pair(s, q);
+    const int rem = L % P;
+    if (rem != 0 || L == 0) a.work[atomicAdd(&hist[bucket(rem)], 1)] = pack_pair(s, full);
+  }
+}
+
+// Wait for an mbarrier phase, or give up. A wait gives up when the CTA-wide
+// abort flag is set, or when it has spun for WAIT_LIMIT_CYCLES; in the second
+// case it sets the flag and reports PKV_DEV_WAIT_TIMEOUT. Either way the
+// caller leaves its loop, so a failure ends the kernel instead of stalling.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              volatile int *abort_flag, int32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      *abort_flag = 1;
+      report(err, PKV_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      "  .reg .pred p;\n"
+      "  mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "  selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bulk copy global -> shared (no tensor map), completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Barrier among the consumer warps only (the scheduler warp keeps running).
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(NCW * 32) : "memory");
+}
+
+// Consumer barrier that also returns the AND of `v` over all consumer threads,
+// so that every consumer warp takes the same exit decision.
+__device__ __forceinline__ bool consumers_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n"
+      "  .reg .pred pin, pout;\n"
+      "  setp.ne.u32 pin, %1, 0;\n"
+      "  bar.red.and.pred pout, 1, %2, pin;\n"
+      "  selp.u32 %0, 1, 0, pout;\n"
+      "}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(NCW * 32)
+      : "memory");
+  return r != 0;
+}
+
+// Merge entries [q0, q1) (at most MERGE_CHUNK) of one (sequence, KV head):
+// for each of its G query heads, o = sum_q 2^(lse_q - lse) o_q with
+// lse = log2 sum_q 2^lse_q. The sources were written by other CTAs; they are
+// read from L2 (ld.global.cg). The result goes to `out` (final), or to chunk
+// entry `dst_idx` of the second-level arrays as (o, lse).
+template <typename T, int D>
+__device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int G,
+                                         const float *src_o, const float *src_lse,
+                                         int src_stride, int q0, int q1, bool final_out,
+                                         int dst_idx) {
+  constexpr int V = D / 4;  // float4 columns per head row
+  T *const out = static_cast<T *>(a.out);
+  const int n_q = q1 - q0;
+  for (int idx = threadIdx.x; idx < G * V; idx += NCW * 32) {
+    const int n = idx / V;
+    const int cv = idx - n * V;
+    const size_t row = (size_t)s * a.num_heads + h * G + n;
+    const float *lse = src_lse + row * src_stride + q0;
+    const float4 *po = reinterpret_cast<const float4 *>(src_o + (row * src_stride + q0) * D) + cv;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NWARPS; ++w) {
-      const float *cw = reinterpret_cast<const float *>(smem_gen + w * NSTAGE * Shape::STAGE_BYTES);
-      M = fmaxf(M, cw[8 * AS + n]);
-    }
-    float num = 0.f, den = 0.f;
+    for (int q = 0; q < MERGE_CHUNK; ++q)
+      if (q < n_q) M = fmaxf(M, __ldcg(lse + q));
+    float W = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < NWARPS; ++w) {
-        const float *cw =
-            reinterpret_cast<const float *>(smem_gen + w * NSTAGE * Shape::STAGE_BYTES);
-        const float f = exp2f(cw[8 * AS + n] - M);
-        num += f * cw[n * AS + d];
-        den += f * cw[8 * AS + 8 + n];
+#pragma unroll 4
+      for (int q = 0; q < n_q; ++q) {
+        const float w = exp2f(__ldcg(lse + q) - M);
+        const float4 v = __ldcg(po + (size_t)q * V);
+        W += w;
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
       }
     }
-    const float o = den > 0.f ? num / den : 0.f;
-    const size_t row = (size_t)s * Hq + h * G + n;
-    if (single) {
-      out[row * D + d] = from_float<T>(o);
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+    if (final_out) {
+      uint2 pk;
+      pk.x = pack2<T>(acc.x, acc.y);
+      pk.y = pack2<T>(acc.z, acc.w);
+      *reinterpret_cast<uint2 *>(out + row * D + 4 * cv) = pk;
     } else {
-      a.ws_o[(row * a.max_parts + p) * D + d] = o;
-      if (d == 0) a.ws_lse[row * a.max_parts + p] = den > 0.f ? M + log2f(den) : -INFINITY;
+      reinterpret_cast<float4 *>(a.ws2_o + (row * a.max_chunks + dst_idx) * D)[cv] = acc;
+      if (cv == 0) a.ws2_lse[row * a.max_chunks + dst_idx] = W > 0.f ? M + log2f(W) : -INFINITY;
     }
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, int NH>
+__global__ void __launch_bounds__(THREADS, 2)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
+  using Shape = TcShape<D, NH>;
+  constexpr int NSTAGE = Shape::NSTAGE;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_abort;
+  const uint32_t raw_addr = smem_addr(smem_raw);
+  const uint32_t smem0 = (raw_addr + 1023u) & ~1023u;  // 128B swizzle wants 1024B alignment
+  uint8_t *const sm = smem_raw + (smem0 - raw_addr);   // generic view of the same base
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int Hq = a.num_heads;
+  const int Hkv = a.num_kv_heads;
+  const int G = Hq / Hkv;
+  const int B = a.block_size;
+
+  const uint32_t bars = smem0 + Shape::BAR_OFF;
+  auto tile_full = [&](int w, int st) { return bars + 8 * (w * NSTAGE + st); };
+  auto item_full = [&](int slot) { return bars + 8 * (NCW * NSTAGE + slot); };
+  auto item_empty = [&](int slot) { return bars + 8 * (NCW * NSTAGE + NSLOT + slot); };
+  ItemDesc *const desc = reinterpret_cast<ItemDesc *>(sm + Shape::DESC_OFF);
+  volatile int *const abort_flag = &s_abort;
+
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < NCW; ++w)
+      for (int st = 0; st < NSTAGE; ++st) mbar_init(tile_full(w, st), 1);
+    for (int sl = 0; sl < NSLOT; ++sl) {
+      mbar_init(item_full(sl), 1);
+      mbar_init(item_empty(sl), NCW);
+    }
+    fence_mbar_init();
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+    // A CTA that starts after some wait already gave up does no work.
+    s_abort = (a.err != nullptr &&
+               *reinterpret_cast<volatile const int32_t *>(a.err) == PKV_DEV_WAIT_TIMEOUT)
+                  ? 1
+                  : 0;
+  }
+  __syncthreads();
+  pdl_wait();  // the work list, counters and everything before the plan are ready
+
+  if (warp == NCW) {
+    // ======================= scheduler warp =======================
+    const long long list_cap = (long long)a.num_seqs * a.max_parts;
+    const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
+    int item = 0;
+    if (lane == 0) item = atomicAdd(&a.sched[0], 1);
+    item = __shfl_sync(FULL_MASK, item, 0);
+    int in_flight = 0;  // posted work / merge descriptors whose completion is not yet handled
+    for (uint32_t it = 0;; ++it) {
+      const int slot = it % NSLOT;
+      ItemDesc &d = desc[slot];
+      int merge_kind = -1, merge_s = 0, merge_h = 0, merge_np = 0, merge_p = 0;
+      if (it >= NSLOT) {
+        if (!__all_sync(FULL_MASK, wait_or_abort(item_empty(slot), ((it / NSLOT) - 1) & 1,
+                                                 abort_flag, a.err)))
+          break;
+        // The consumers are done with the slot's previous descriptor: publish
+        // a finished partition / chunk result and post the merge it completes.
+        const int pk = d.kind;
+        if (pk == KIND_WORK || pk == KIND_MERGE_CHUNK || pk == KIND_MERGE_FINAL) --in_flight;
+        const int np = d.nparts;
+        const int nchunks = (np + MERGE_CHUNK - 1) / MERGE_CHUNK;
+        int next_kind = -1, next_p = 0;
+        if (lane == 0 && ((pk == KIND_WORK && np > 1) || pk == KIND_MERGE_CHUNK)) {
+          __threadfence();
+          if (pk == KIND_WORK) {
+            const int ch = d.p / MERGE_CHUNK;
+            const int ch_size = min(MERGE_CHUNK, np - ch * MERGE_CHUNK);
+            const int t = atomicAdd(&a.merge_cnt[(d.s * Hkv + d.h) * a.max_chunks + ch], 1);
+            if (t == ch_size - 1) {
+              next_kind = nchunks == 1 ? KIND_MERGE_FINAL : KIND_MERGE_CHUNK;
+              next_p = ch;
+            }
+          } else {
+            const int t = atomicAdd(&a.merge_cnt2[d.s * Hkv + d.h], 1);
+            if (t == nchunks - 1) next_kind = KIND_MERGE_FINAL;
+          }
+          if (next_kind >= 0) __threadfence();
+        }
+        next_kind = __shfl_sync(FULL_MASK, next_kind, 0);
+        if (next_kind >= 0) {
+          merge_kind = next_kind;
+          merge_s = d.s;
+          merge_h = d.h;
+          merge_np = np;
+          merge_p = __shfl_sync(FULL_MASK, next_p, 0);
+        }
+      }
+      __syncwarp();  // every lane has read the old descriptor before it is rewritten
+      if (merge_kind >= 0) {
+        if (lane == 0) {
+          d.kind = merge_kind;
+          d.s = merge_s;
+          d.h = merge_h;
+          d.p = merge_p;
+          d.nparts = merge_np;
+          d.n_tiles = 0;
+          mbar_arrive(item_full(slot));
+        }
+        ++in_flight;
+        continue;
+      }
+      if (item >= total_items) {
+        // No new work: keep the ring turning (no-op descriptors) until every
+        // posted item has completed and produced its merge tasks, then stop.
+        if (lane == 0) {
+          d.kind = in_flight == 0 ? KIND_END : KIND_NOP;
+          d.n_tiles = 0;
+          mbar_arrive(item_full(slot));
+        }
+        if (in_flight == 0) break;
+        continue;
+      }
+      int next = 0;
+      if (lane == 0) next = atomicAdd(&a.sched[0], 1);  // consumed at the end of this item
+
+      const uint32_t pr = a.work[item / Hkv];
+      const int h = item - (item / Hkv) * Hkv;
+      const int s = min(static_cast<int>(pr >> 16), a.num_seqs - 1);
+      const int p = static_cast<int>(pr & 0xffffu);
+      const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, B,
+                                  lane == 0 ? a.err : nullptr);
+      const int t_begin = p * a.part_tokens;
+      const int t_end = min(L, t_begin + a.part_tokens);
+      const int n_tiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
+      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
+      for (int t = lane; t < n_tiles && t < DESC_TILES; t += 32)
+        d.ids[t] = bt[(t_begin + t * TILE) / B];
+      if (lane == 0) {
+        d.kind = KIND_WORK;
+        d.s = s;
+        d.p = p;
+        d.h = h;
+        d.L = L;
+        d.n_tiles = n_tiles;
+        d.nparts = (L + a.part_tokens - 1) / a.part_tokens;
+      }
+      __syncwarp();  // every lane's ids precede lane 0's release below
+      if (lane == 0) {
+        const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
+        mbar_arrive_expect_tx(item_full(slot), qbytes);
+        if (qbytes)
+          bulk_load(smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES,
+                    static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
+                    item_full(slot));
+      }
+      ++in_flight;
+      item = __shfl_sync(FULL_MASK, next, 0);
+    }
+    return;
+  }
+
+  // ======================= consumer warps =======================
+  const int g = lane >> 2;  // mma group id (row of A / column of B)
+  const int c = lane & 3;   // thread in group
+  const float sl2 = a.scale_log2;
+  T *const out = static_cast<T *>(a.out);
+  const int mi = lane >> 3;                      // ldmatrix: lane feeds row (lane & 7)
+  const int vr = (lane & 7) + ((mi >> 1) << 3);  //   of matrix mi; token row in the tile
+  constexpr int AS = Shape::ACC_STRIDE;
+  const uint32_t ring = smem0 + warp * NSTAGE * Shape::STAGE_BYTES;
+  const int total_rows = a.num_blocks * Hkv * B;
+  float *const comb = reinterpret_cast<float *>(sm + Shape::COMBINE_OFF);
+  float *const cw_me = comb + warp * Shape::CW_FLOATS;  // this warp's combine rows
+  float *const scales = comb + NCW * Shape::CW_FLOATS;  // [NH][NCW] weights, [NH] lse
+
+  // Issue side of this warp's ring. It walks the same descriptor sequence as
+  // the consume side but runs up to NSTAGE tiles ahead, across item boundaries.
+  uint32_t issued = 0, done = 0;  // tiles of this warp issued / consumed so far
+  uint32_t bad_mask = 0;          // bit st: the tile in stage st had an invalid block id
+  uint32_t is_it = 0;             // descriptor being issued
+  int is_j = 0, is_ntw = 0, is_h = 0, is_tbegin = 0, is_s = 0;
+  bool is_ready = false, is_end = false;
+
+  // Issue this warp's next tiles while fewer than NSTAGE are in flight. With
+  // `must`, block (bounded) for the next descriptor when nothing is in flight.
+  auto pump = [&](bool must) {
+    while (issued - done < (uint32_t)NSTAGE && !is_end) {
+      if (!is_ready) {
+        const int sl = is_it % NSLOT;
+        const uint32_t par = (is_it / NSLOT) & 1;
+        bool ok;
+        if (must && issued == done)
+          ok = wait_or_abort(item_full(sl), par, abort_flag, a.err);
+        else
+          ok = mbar_test(item_full(sl), par);
+        if (!__all_sync(FULL_MASK, ok)) return;
+        const ItemDesc &d = desc[sl];
+        if (d.kind == KIND_END) {
+          is_end = true;
+          return;
+        }
+        const int nt = d.kind == KIND_WORK ? d.n_tiles : 0;
+        is_s = d.s;
+        is_h = d.h;
+        is_tbegin = d.p * a.part_tokens;
+        is_ntw = warp < nt ? (nt - warp + NCW - 1) / NCW : 0;
+        is_j = 0;
+        is_ready = true;
+      }
+      if (is_j >= is_ntw) {
+        ++is_it;
+        is_ready = false;
+        continue;
+      }
+      const int tile = warp + is_j * NCW;
+      const int tok0 = is_tbegin + tile * TILE;
+      const int phys = tile < DESC_TILES ? desc[is_it % NSLOT].ids[tile]
+                                         : a.block_tables[(size_t)is_s * a.max_blocks + tok0 / B];
+      const int st = issued % NSTAGE;
+      const bool bad = phys < 0 || phys >= a.num_blocks;
+      bad_mask = bad ? (bad_mask | (1u << st)) : (bad_mask & ~(1u << st));
+      if (lane == 0) {
+        int y;
+        if (bad) {
+          report(a.err, PKV_DEV_BAD_BLOCK);
+          y = total_rows;  // wholly out of bounds: TMA fills zeros
+        } else {
+          y = (phys * Hkv + is_h) * B + (tok0 % B);
+        }
+        const uint32_t bar = tile_full(warp, st);
+        const uint32_t kdst = ring + st * Shape::STAGE_BYTES;
+        const uint32_t vdst = kdst + Shape::KT_BYTES;
+        mbar_arrive_expect_tx(bar, Shape::STAGE_BYTES);
+#pragma unroll
+        for (int hh = 0; hh < Shape::HALVES; ++hh) {
+          tma_load_2d(kdst + hh * HALF_BYTES, &tmK, hh * BOX_COLS, y, bar);
+          tma_load_2d(vdst + hh * HALF_BYTES, &tmV, hh * BOX_COLS, y, bar);
+        }
+      }
+      ++issued;
+      ++is_j;
+    }
+  };
+
+  for (uint32_t it = 0;; ++it) {
+    const int slot = it % NSLOT;
+    const bool got = wait_or_abort(item_full(slot), (it / NSLOT) & 1, abort_flag, a.err);
+    if (!consumers_all(got)) break;
+    const ItemDesc &dref = desc[slot];
+    const int kind = dref.kind;
+    if (kind == KIND_END) break;  // the same descriptor for every consumer: a uniform exit
+    if (kind != KIND_WORK) {
+      const int np = dref.nparts;
+      if (kind == KIND_MERGE_CHUNK) {
+        const int q0 = dref.p * MERGE_CHUNK;
+        merge_range<T, D>(a, dref.s, dref.h, G, a.ws_o, a.ws_lse, a.max_parts, q0,
+                          min(np, q0 + MERGE_CHUNK), false, dref.p);
+      } else if (kind == KIND_MERGE_FINAL) {
+        if (np <= MERGE_CHUNK)
+          merge_range<T, D>(a, dref.s, dref.h, G, a.ws_o, a.ws_lse, a.max_parts, 0, np, true, 0);
+        else
+          merge_range<T, D>(a, dref.s, dref.h, G, a.ws2_o, a.ws2_lse, a.max_chunks, 0,
+                            (np + MERGE_CHUNK - 1) / MERGE_CHUNK, true, 0);
+      }
+      pump(false);
+      consumers_sync();  // the descriptor is read by all before the slot is handed back
+      if (lane == 0) mbar_arrive(item_empty(slot));
+      continue;
+    }
+    const int s = dref.s, p = dref.p, h = dref.h, L = dref.L, n_tiles = dref.n_tiles;
+    const int nparts = dref.nparts;
+    const int t_begin = p * a.part_tokens;
+    const int nt_w = warp < n_tiles ? (n_tiles - warp + NCW - 1) / NCW : 0;
+
+    pump(false);  // top up the ring (this item, and beyond)
+
+    // Q^T as the B operand: lane (g, c) holds head g's elements
+    // 8*Lc .. 8*Lc+7 for logical chunk Lc(c, j) = (j/2)*8 + 2c + (j%2).
+    uint4 qf[D / 32];
+    {
+      const uint32_t qrow = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES + g * D * 2;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const int Lc = (j >> 1) * 8 + 2 * c + (j & 1);
+        qf[j] = (g < G && n_tiles > 0) ? lds128(qrow + Lc * 16) : make_uint4(0, 0, 0, 0);
+      }
+    }
+
+    float acc[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY;  // reference max of heads 2c, 2c+1 (base-2 units)
+    float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
+    bool aborted = false;
+
+    for (int j = 0; j < nt_w; ++j) {
+      if (issued == done) pump(true);
+      const int st = done % NSTAGE;
+      if (issued == done ||
+          !__all_sync(FULL_MASK, wait_or_abort(tile_full(warp, st), (done / NSTAGE) & 1,
+                                               abort_flag, a.err))) {
+        aborted = true;
+        break;
+      }
+      const uint32_t ks = ring + st * Shape::STAGE_BYTES;
+      const uint32_t vs = ks + Shape::KT_BYTES;
+      const int tok0 = t_begin + (warp + j * NCW) * TILE;
+      const int valid = min(TILE, L - tok0);
+      const bool bad = (bad_mask >> st) & 1u;
+
+      if (valid < TILE && !bad) {
+        // Tokens past the context length: their V rows may hold anything
+        // (NaN included); zero them so P*V stays finite.
+        const int nchunks = (TILE - valid) * 8 * Shape::HALVES;
+        for (int e = lane; e < nchunks; e += 32) {
+          const int r = valid + e / (8 * Shape::HALVES);
+          const int rem = e % (8 * Shape::HALVES);
+          sts128_zero(vs + (rem >> 3) * HALF_BYTES + r * 128 + (rem & 7) * 16);
+        }
+        fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
+        __syncwarp();
+      }
+
+      // ---- scores: S^T = K . Q^T (two independent accumulation chains) ----
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int jj = 0; jj < D / 32; ++jj) {
+        const int Lc = (jj >> 1) * 8 + 2 * c + (jj & 1);
+        const uint32_t rowg = ks + (Lc >> 3) * HALF_BYTES + g * 128 + (((Lc & 7) ^ g) << 4);
+        const uint4 ka = lds128(rowg);            // token g
+        const uint4 kb = lds128(rowg + 8 * 128);  // token g + 8 (same swizzle phase)
+        mma16816<T>(sa, ka.x, kb.x, ka.y, kb.y, qf[jj].x, qf[jj].y);
+        mma16816<T>(sb, ka.z, kb.z, ka.w, kb.w, qf[jj].z, qf[jj].w);
+      }
+
+      // ---- online softmax (heads 2c, 2c+1; tokens g, g+8) ----
+      const bool ok0 = !bad && g < valid;
+      const bool ok1 = !bad && g + 8 < valid;
+      const float x0 = ok0 ? (sa[0] + sb[0]) * sl2 : -INFINITY;
+      const float x1 = ok0 ? (sa[1] + sb[1]) * sl2 : -INFINITY;
+      const float x2 = ok1 ? (sa[2] + sb[2]) * sl2 : -INFINITY;
+      const float x3 = ok1 ? (sa[3] + sb[3]) * sl2 : -INFINITY;
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
+      }
+      // Lazy reference max: keep it unless this tile exceeds it by more than
+      // 2^RESCALE_SLACK (then p <= 2^8 stays well inside fp32/bf16/fp16 range).
+      const bool up0 = mx0 > m0 + RESCALE_SLACK, up1 = mx1 > m1 + RESCALE_SLACK;
+      if (__any_sync(FULL_MASK, up0 || up1)) {
+        const float mn0 = up0 ? mx0 : m0, mn1 = up1 ? mx1 : m1;
+        const float al0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - mn0);
+        const float al1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mn1);
+        l0 *= al0;
+        l1 *= al1;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          acc[mt][0] *= al0;
+          acc[mt][1] *= al1;
+          acc[mt][2] *= al0;
+          acc[mt][3] *= al1;
+        }
+        m0 = mn0;
+        m1 = mn1;
+      }
+      const float mu0 = m0 == -INFINITY ? 0.f : m0;
+      const float mu1 = m1 == -INFINITY ? 0.f : m1;
+      const float p0 = ex2_approx(x0 - mu0), p1 = ex2_approx(x1 - mu1);
+      const float p2 = ex2_approx(x2 - mu0), p3 = ex2_approx(x3 - mu1);
+      l0 += p0 + p2;
+      l1 += p1 + p3;
+
+      // P^T as the B operand: transpose the (token, head) fragment pairs.
+      const uint32_t pb0 = movmatrix_trans(pack2<T>(p0, p1));  // tokens 0..7
+      const uint32_t pb1 = movmatrix_trans(pack2<T>(p2, p3));  // tokens 8..15
+
+      // ---- O^T += V^T . P^T ----
+      const uint32_t vrow = vs + vr * 128;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int chunk = 2 * mt + (mi & 1);
+        const uint32_t addr = vrow + (chunk >> 3) * HALF_BYTES + (((chunk & 7) ^ (vr & 7)) << 4);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_trans(addr, r0, r1, r2, r3);
+        mma16816<T>(acc[mt], r0, r1, r2, r3, pb0, pb1);
+      }
+      __syncwarp();  // every lane is done with this stage before it is refilled
+      ++done;
+      pump(false);
+    }
+
+    // Full per-warp sums: add the 8 lanes that share a head pair.
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(FULL_MASK, l0, off);
+      l1 += __shfl_xor_sync(FULL_MASK, l1, off);
+    }
+
+    // ---- combine the consumer warps ----
+    // 1) each warp stores its unnormalised rows and (max, sum) per head
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      if (2 * c < NH) {
+        cw_me[(2 * c) * AS + 16 * mt + g] = acc[mt][0];
+        cw_me[(2 * c) * AS + 16 * mt + g + 8] = acc[mt][2];
+      }
+      if (2 * c + 1 < NH) {
+        cw_me[(2 * c + 1) * AS + 16 * mt + g] = acc[mt][1];
+        cw_me[(2 * c + 1) * AS + 16 * mt + g + 8] = acc[mt][3];
+      }
+    }
+    if (g == 0) {
+      if (2 * c < NH) {
+        cw_me[NH * AS + 2 * c] = m0;
+        cw_me[NH * AS + NH + 2 * c] = l0;
+      }
+      if (2 * c + 1 < NH) {
+        cw_me[NH * AS + 2 * c + 1] = m1;
+        cw_me[NH * AS + NH + 2 * c + 1] = l1;
+      }
+    }
+    consumers_sync();
+    // 2) per head: warp weights 2^(m_w - M) / sum, and the log2-sum-exp
+    if (threadIdx.x < G) {
+      const int n = threadIdx.x;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) M = fmaxf(M, comb[w * Shape::CW_FLOATS + NH * AS + n]);
+      float f[NCW], den = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float mw = comb[w * Shape::CW_FLOATS + NH * AS + n];
+        f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        den += f[w] * comb[w * Shape::CW_FLOATS + NH * AS + NH + n];
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) scales[n * NCW + w] = f[w] * inv;
+      scales[NH * NCW + n] = den > 0.f ? M + log2f(den) : -INFINITY;
+    }
+    consumers_sync();
+    // 3) outputs
+    const bool single = nparts <= 1;
+    for (int idx = threadIdx.x; idx < G * D; idx += NCW * 32) {
+      const int n = idx / D;
+      const int dd = idx - n * D;
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w)
+        o += scales[n * NCW + w] * comb[w * Shape::CW_FLOATS + n * AS + dd];
+      const size_t row = (size_t)s * Hq + h * G + n;
+      if (single) {
+        out[row * D + dd] = from_float<T>(o);
+      } else {
+        a.ws_o[(row * a.max_parts + p) * D + dd] = o;
+        if (dd == 0) a.ws_lse[row * a.max_parts + p] = scales[NH * NCW + n];
+      }
+    }
+    // Everyone is done with the combine area and this item's descriptor/q;
+    // the vote makes a stop (after a wait gave up anywhere) uniform. Handing
+    // the slot back also publishes this item's global writes to the scheduler.
+    const bool go_on = consumers_all(!aborted && *abort_flag == 0);
+    if (lane == 0) mbar_arrive(item_empty(slot));
+    if (!go_on) break;
+  }
+}
+
+int sm_count_for_current_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+template <typename T, int D, int NH>
 cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                       cudaStream_t stream) {
-  using Shape = TcShape<D>;
-  auto kern = decode_tc_kernel<T, D>;
+  using Shape = TcShape<D, NH>;
+  auto kern = decode_tc_kernel<T, D, NH>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.max_parts, a.num_kv_heads, a.num_seqs);
-  kern<<<grid, NWARPS * 32, Shape::SMEM_BYTES, stream>>>(tmK, tmV, a);
-  return cudaGetLastError();
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, Shape::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const long long max_items = (long long)a.num_seqs * a.max_parts * a.num_kv_heads;
+  long long grid = (long long)sm_count_for_current_device() * per_sm;
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+
+  plan_kernel<<<1, PLAN_THREADS, 0, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // Programmatic dependent launch: the decode CTAs start (barrier set-up,
+  // descriptor prefetch) while the plan runs, and wait for it before reading
+  // the work list.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, a);
+}
+
+template <typename T>
+cudaError_t launch_tc_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                        cudaStream_t stream) {
+  const int G = a.num_heads / a.num_kv_heads;
+  if (a.head_dim == 64)
+    return G <= 4 ? launch_tc<T, 64, 4>(a, tmK, tmV, stream)
+                  : launch_tc<T, 64, 8>(a, tmK, tmV, stream);
+  return G <= 4 ? launch_tc<T, 128, 4>(a, tmK, tmV, stream)
+                : launch_tc<T, 128, 8>(a, tmK, tmV, stream);
 }
 
 }  // namespace
 
 size_t decode_tc_smem_bytes(int head_dim) {
-  return head_dim == 64 ? TcShape<64>::SMEM_BYTES : TcShape<128>::SMEM_BYTES;
+  return head_dim == 64 ? TcShape<64, 8>::SMEM_BYTES : TcShape<128, 8>::SMEM_BYTES;
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t stream) {
-  if (dtype == PKV_BF16) {
-    if (a.head_dim == 64) return launch_tc<__nv_bfloat16, 64>(a, tmK, tmV, stream);
-    return launch_tc<__nv_bfloat16, 128>(a, tmK, tmV, stream);
-  }
-  if (a.head_dim == 64) return launch_tc<__half, 64>(a, tmK, tmV, stream);
-  return launch_tc<__half, 128>(a, tmK, tmV, stream);
+  if (dtype == PKV_BF16) return launch_tc_t<__nv_bfloat16>(a, tmK, tmV, stream);
+  return launch_tc_t<__half>(a, tmK, tmV, stream);
 }
 
 }  // namespace pkv

@@ -29,8 +29,31 @@ struct DecodeArgs {
   int max_parts;       // partitions of the longest allowed context
   float scale_log2;    // scale * log2(e): scores are kept in base-2 units
   int32_t *err;        // nullable device error word
+  // Work list of the persistent decode kernel (written by the plan kernel):
+  uint32_t *work;      // [<= S*max_parts] (seq << 16 | partition), full partitions first
+  int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries
+  // Partition merging (split contexts). Partitions are merged in chunks of
+  // MERGE_CHUNK; a context with more than one chunk is merged in two levels.
+  int32_t *merge_cnt;  // [S*Hkv][max_chunks] finished partitions per chunk; zeroed by the plan
+  int32_t *merge_cnt2; // [S*Hkv] finished chunk merges; zeroed by the plan
+  float *ws2_o;        // [S][Hq][max_chunks][D] chunk results (normalised), or null
+  float *ws2_lse;      // [S][Hq][max_chunks] chunk log2-sum-exp, or null
+  int max_chunks;      // ceil(max_parts / MERGE_CHUNK)
 };
 
+constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
+
+// Decode workspace, in order: scheduling words (256 B), the work list, then
+// (only when a context can span several partitions) the merge counters, the
+// partition outputs with their log2-sum-exp values, and (only when a context
+// can span several merge chunks) the chunk results. Each region is 256-byte
+// aligned.
+struct WorkspaceLayout {
+  size_t sched_off, work_off, cnt_off, cnt2_off, o_off, lse_off, o2_off, lse2_off, total;
+};
+WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long long max_parts);
+
+// Plan + persistent decode (+ merge when split) for fp16 / bf16.
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t stream);
 cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream);

@@ -53,12 +53,19 @@ def test_status_strings(lib):
 
 def test_workspace_arithmetic(lib):
     f = lib.pkv_decode_workspace_bytes
-    assert f(8, 32, 128, 512, 512) == 0          # one partition: no workspace
-    assert f(8, 32, 128, 100, 0) == 0            # unsplit
-    # 8 seqs x 32 heads x 256 partitions: fp32 outputs [..][128] + one lse each
-    assert f(8, 32, 128, 131072, 512) == 8 * 32 * 256 * 128 * 4 + 8 * 32 * 256 * 4
-    # 33 tokens in 16-token partitions = 3 partitions; regions are 256-byte aligned
-    assert f(1, 1, 64, 33, 16) == 3 * 64 * 4 + 256
+    # scheduling words (256 B) + work list (one uint32 per (seq, partition)),
+    # each region rounded up to 256 B
+    assert f(8, 32, 128, 512, 512) == 256 + 256   # one partition: no partials
+    assert f(8, 32, 128, 100, 0) == 256 + 256     # unsplit
+    # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16): chunk and
+    # final merge counters, fp32 partition outputs + lse, chunk results + lse
+    S, Hq, D, P, C = 8, 32, 128, 256, 16
+    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 4 + S * Hq * C * 4 + S * Hq * 4
+                                        + S * Hq * P * D * 4 + S * Hq * P * 4
+                                        + S * Hq * C * D * 4 + S * Hq * C * 4)
+    # 33 tokens in 16-token partitions = 3 partitions, one merge chunk
+    assert f(1, 1, 64, 33, 16) == 256 + 256 + 256 + 256 + 3 * 64 * 4 + 256
+    assert f(0, 32, 128, 512, 512) == 0
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below is rejected first
