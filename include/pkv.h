@@ -126,6 +126,46 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
                       int dtype, int partition_size, void *workspace, size_t workspace_bytes,
                       int32_t *err, void *stream);
 
+/* Size of the library-owned scratch array used by paged_attn_decode_static_ws. */
+#define PKV_STATIC_WS_BYTES (64u * 1024u * 1024u)
+
+/*
+ * paged_attn_decode_static_ws - paged_attn_decode for callers that cannot
+ * allocate device memory when they decode. The pages describe nothing like
+ * it; it is a convenience of this library.
+ *
+ * Who needs it: a serving engine that reserved (almost) all device memory for
+ * its KV block pool at start-up, where a later cudaMalloc for split-context
+ * workspace may fail or bypass the engine's allocator. Also hosts that allow
+ * no device allocation after initialisation, because cudaMalloc can
+ * synchronise the device and takes an unpredictable time.
+ *
+ * Arguments and results are those of paged_attn_decode, without workspace and
+ * workspace_bytes. The workspace instead comes from a fixed array of
+ * PKV_STATIC_WS_BYTES (64 MiB) inside the library. This call allocates
+ * nothing itself: no cudaMalloc, cudaFree or allocating library call.
+ *
+ * Limits and sharing:
+ *  - If pkv_decode_workspace_bytes(...) for the arguments exceeds
+ *    PKV_STATIC_WS_BYTES, the call returns PKV_EUNSUPPORTED and enqueues
+ *    nothing; use paged_attn_decode with your own workspace then.
+ *  - Each GPU holds its own copy of the array from the first call made on it
+ *    until the process exits.
+ *  - The first call on a device looks up that copy's address (one
+ *    cudaGetSymbolAddress) with the device current. Make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; the decode resets what it needs on every call. Calls whose
+ *    GPU work can overlap in time (different streams without ordering between
+ *    them) race on the array and give wrong results; order them.
+ */
+int paged_attn_decode_static_ws(void *out, const void *q, const void *k_pool, const void *v_pool,
+                                const int32_t *block_tables, const int32_t *context_lens,
+                                int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                int block_size, int max_blocks_per_seq, int num_blocks,
+                                int max_context_len, float scale, int dtype, int partition_size,
+                                int32_t *err, void *stream);
+
 /*
  * kv_cache_append - write new tokens' K/V into their slots.
  *
