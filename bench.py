@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--workload", default="llama8b_gqa_b256")
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="keep only the first sequences of the workload (small profiling cases)")
+    ap.add_argument("--partition-size", type=int, default=None,
+                    help="tokens per split-context partition (default: the workload's)")
     ap.add_argument("--soak-seconds", type=float, default=2.0,
                     help="back-to-back steps before the timed region (clock sampling, warm clocks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -292,6 +294,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs)
+    if args.partition_size is not None:
+        case.partition_size = args.partition_size
     stream = torch.cuda.current_stream(dev)
 
     S, Hq, D = case.num_seqs, case.num_heads, case.head_dim
