@@ -171,6 +171,30 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic (one process per GPU; no data collective)
+# ---------------------------------------------------------------------------
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling): same workload, another seed."""
+    return int(base_seed) + 1000 * int(rank)
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_gbs(bytes_per_rank: int, world: int, seconds: float) -> float:
+    """Aggregate throughput: the bytes every rank moved / the slowest rank's time."""
+    return bytes_per_rank * world / seconds / 1e9
+
+
+# ---------------------------------------------------------------------------
 # the reference arm: the CPU oracle, timed on the host cores
 # ---------------------------------------------------------------------------
 
@@ -293,7 +317,9 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs)
+    from pkv_inputs.workloads import WORKLOADS
+    case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
+                     seed=rank_seed(WORKLOADS[args.workload]["seed"], rank))
     if args.partition_size is not None:
         case.partition_size = args.partition_size
     stream = torch.cuda.current_stream(dev)
@@ -357,14 +383,10 @@ def run_ours(args, rank, world, local_rank):
 
     ms = start.elapsed_time(end) / args.steps
     dec_ms = statistics.mean(a.elapsed_time(b) for a, b in dec_events)
-    if world > 1:
-        t = torch.tensor([ms, dec_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(t[0]), float(t[1])
+    ms, dec_ms = max_over_ranks([ms, dec_ms], dev)
 
     dec_bytes, app_bytes = step_bytes(case)
-    total_bytes = (dec_bytes + app_bytes) * world
-    value = total_bytes / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(dec_bytes + app_bytes, world, ms * 1e-3)
 
     # ---- end to end: host buffers, copies inside the timed region ----
     host_in = {k: getattr(case, k).cpu().pin_memory()
@@ -392,12 +414,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = total_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
+    e2e_value = whole_job_gbs(dec_bytes + app_bytes, world, e2e_ms * 1e-3)
 
     torch.cuda.synchronize()
     if int(err.item()) != 0:
