@@ -284,7 +284,11 @@ def run_reference(args, rank, world):
 
 def config_block(case, workload, n_gpus):
     from pkv_inputs.workloads import WORKLOADS
-    desc = WORKLOADS.get(workload, {}).get("desc", workload)
+    desc = WORKLOADS.get(workload, {}).get(
+        "desc", "shared prefix / parallel sampling: 16 prompts x 6 samples, 40 heads MHA, "
+                "head_dim 128, fp16, block 16, prompt 1000 tokens shared through refcounted "
+                "blocks, CoW copy of the partial block, then 64 divergent decode tokens "
+                "(the timed step is the 64th)" if workload == "shared_prefix" else workload)
     return {
         "workload": workload, "desc": desc, "num_seqs_per_gpu": case.num_seqs,
         "num_heads": case.num_heads, "num_kv_heads": case.num_kv_heads,
@@ -304,6 +308,68 @@ def config_block(case, workload, n_gpus):
 # our arm
 # ---------------------------------------------------------------------------
 
+def build_bench_case(args, dev, rank):
+    """The step's inputs, plus extra report fields for special workloads."""
+    import torch
+    from pkv_inputs import make_case
+    from pkv_inputs.workloads import WORKLOADS, DecodeCase, make_shared_prefix_case
+    if args.workload != "shared_prefix":
+        case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
+                         seed=rank_seed(WORKLOADS[args.workload]["seed"], rank))
+        return case, {}
+    # 16 prompts x 6 samples sharing refcounted prompt blocks: the copy-on-write
+    # block copies run once, then the samples decode 64 divergent tokens. The
+    # timed step is the last one (append + decode at context 1064).
+    import paged_kv_cache_387_b200 as pkv
+    sp = make_shared_prefix_case(device=dev, seed=rank_seed(391, rank))
+    pairs = sp.cow_pairs
+    pkv.kv_block_copy(sp.k_pool, sp.v_pool, pairs)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    reps = 20
+    for _ in range(reps):  # idempotent: the same copies again
+        pkv.kv_block_copy(sp.k_pool, sp.v_pool, pairs)
+    b.record()
+    torch.cuda.synchronize()
+    copy_ms = a.elapsed_time(b) / reps
+    blk = sp.num_kv_heads * sp.block_size * sp.head_dim * sp.k_pool.element_size()
+    copy_bytes = 2 * 2 * blk * int(pairs.shape[0])  # read + write, K and V
+    last = len(sp.steps) - 1
+    for k in range(last):
+        _, kn, vn = sp.step_tokens(k)
+        pkv.kv_cache_append(sp.k_pool, sp.v_pool, kn, vn, sp.steps[k]["slot_mapping"])
+    q, kn, vn = sp.step_tokens(last)
+    st = sp.steps[last]
+    case = DecodeCase(name="shared_prefix", q=q, k_pool=sp.k_pool, v_pool=sp.v_pool,
+                      block_tables=st["block_tables"], context_lens=st["context_lens"],
+                      num_heads=sp.num_heads, num_kv_heads=sp.num_kv_heads,
+                      head_dim=sp.head_dim, block_size=sp.block_size, scale=sp.scale,
+                      partition_size=sp.partition_size, k_new=kn, v_new=vn,
+                      slot_mapping=st["slot_mapping"])
+    # unique K/V bytes: the shared full prompt blocks once per prompt, plus every
+    # sample's own blocks
+    bt = st["block_tables"].cpu()
+    lens = st["context_lens"].cpu()
+    per_tok = 2 * sp.num_kv_heads * sp.head_dim * sp.k_pool.element_size()
+    seen, unique_tokens = set(), 0
+    for s_ in range(bt.shape[0]):
+        L = int(lens[s_])
+        for j in range(-(-L // sp.block_size)):
+            phys = int(bt[s_, j])
+            if phys not in seen:
+                seen.add(phys)
+                unique_tokens += min(sp.block_size, L - j * sp.block_size)
+    extras = {"block_copy": {"pairs": int(pairs.shape[0]), "ms": copy_ms,
+                             "GB/s": copy_bytes / (copy_ms * 1e-3) / 1e9,
+                             "bytes": copy_bytes},
+              "shared_prefix": {"logical_kv_bytes": int(lens.sum()) * per_tok,
+                                "unique_kv_bytes": unique_tokens * per_tok,
+                                "prompts": sp.num_prompts, "samples": sp.samples,
+                                "note": "value/roofline count logical bytes; blocks shared "
+                                        "by the samples of a prompt are read from L2"}}
+    return case, extras
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -317,9 +383,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    from pkv_inputs.workloads import WORKLOADS
-    case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
-                     seed=rank_seed(WORKLOADS[args.workload]["seed"], rank))
+    case, extras = build_bench_case(args, dev, rank)
     if args.partition_size is not None:
         case.partition_size = args.partition_size
     stream = torch.cuda.current_stream(dev)
@@ -330,7 +394,12 @@ def run_ours(args, rank, world, local_rank):
     ws_bytes = pkv.decode_workspace_bytes(S, Hq, D, mcl, case.partition_size)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    launches_per_step = 1 + 1 + (1 if ws_bytes > 0 else 0)
+    # append, then plan + decode (16-bit; the merge is fused into the decode),
+    # or decode + merge kernel when split (fp32)
+    if case.q.dtype == torch.float32:
+        launches_per_step = 2 + (1 if mcl > case.partition_size > 0 else 0)
+    else:
+        launches_per_step = 3
 
     def decode(c, o):
         pkv.paged_attn_decode(o, c.q, c.k_pool, c.v_pool, c.block_tables, c.context_lens,
@@ -389,32 +458,84 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_gbs(dec_bytes + app_bytes, world, ms * 1e-3)
 
     # ---- end to end: host buffers, copies inside the timed region ----
-    host_in = {k: getattr(case, k).cpu().pin_memory()
-               for k in ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")}
-    dev_in = {k: getattr(case, k) for k in host_in}
-    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    # Every step copies its own inputs from pinned host memory and its output
+    # back, as a serving loop does. The copies run on two copy streams, with
+    # double-buffered device inputs/outputs, so step i+1's upload and step
+    # i-1's download overlap step i's kernels.
+    names = ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")
+    host_in = {k: getattr(case, k).cpu().pin_memory() for k in names}
+    dev_sets = [{k: torch.empty_like(getattr(case, k)) for k in names} for _ in range(2)]
+    outs = [torch.empty_like(out) for _ in range(2)]
+    host_outs = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_outs[0].numel() * host_outs[0].element_size()
+    h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    out_ready = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for k, t in host_in.items():
-            dev_in[k].copy_(t, non_blocking=True)
-        step()
-        host_out.copy_(out, non_blocking=True)
+    def run_step(inp, o):
+        pkv.kv_cache_append(case.k_pool, case.v_pool, inp["k_new"], inp["v_new"],
+                            inp["slot_mapping"], err=err)
+        pkv.paged_attn_decode(o, inp["q"], case.k_pool, case.v_pool, inp["block_tables"],
+                              inp["context_lens"], case.scale, mcl,
+                              partition_size=case.partition_size, workspace=ws, err=err)
 
-    for _ in range(3):
-        e2e_step()
+    def e2e_steps(n, start_event=None):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d_stream):
+                if i >= 2:
+                    h2d_stream.wait_event(in_free[b])
+                elif start_event is not None:
+                    h2d_stream.wait_event(start_event)
+                for k in names:
+                    dev_sets[b][k].copy_(host_in[k], non_blocking=True)
+                in_ready[b].record(h2d_stream)
+            stream.wait_event(in_ready[b])
+            if i >= 2:
+                stream.wait_event(out_free[b])
+            run_step(dev_sets[b], outs[b])
+            in_free[b].record(stream)
+            out_ready[b].record(stream)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(out_ready[b])
+                host_outs[b].copy_(outs[b], non_blocking=True)
+                out_free[b].record(d2h_stream)
+        last = torch.cuda.Event()
+        last.record(d2h_stream)
+        stream.wait_event(last)
+
+    e2e_steps(3)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_steps(args.steps, start_event=e0)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
+
+    # the copy engines' own rates for this step's transfer sizes (diagnostic)
+    def copy_gbs(dst, src, nbytes, reps=20):
+        for _ in range(3):
+            dst.copy_(src, non_blocking=True)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            dst.copy_(src, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return nbytes * reps / (a.elapsed_time(b) * 1e-3) / 1e9
+    flat_h = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
+    flat_d = torch.empty(h2d, dtype=torch.uint8, device=dev)
+    h2d_gbs = copy_gbs(flat_d, flat_h, h2d)
+    d2h_gbs = copy_gbs(host_outs[0], outs[0], d2h)
+    del flat_h, flat_d
     e2e_value = whole_job_gbs(dec_bytes + app_bytes, world, e2e_ms * 1e-3)
 
     torch.cuda.synchronize()
@@ -422,7 +543,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error word set: {pkv.device_error_message(int(err.item()))}")
 
     contiguous = None
-    if args.contiguous:
+    if args.contiguous and args.workload != "shared_prefix":
         ccase = make_case(args.workload, device=dev, with_append=False, placement="identity",
                           num_seqs=args.num_seqs)
         cout = torch.empty_like(ccase.q)
@@ -459,18 +580,26 @@ def run_ours(args, rank, world, local_rank):
         "seq_steps_per_s": S * world / (ms * 1e-3),
         "pct_of_hbm_peak": {"of_spec_8000_gbs": value / (HBM_SPEC_GBS * world),
                             f"of_{peak_kind}_{peak:.0f}_gbs": value / (peak * world)},
-        "roofline": {"kernel": "paged_attn_decode (decode_tc_kernel + merge_kernel)",
+        "roofline": {"kernel": "paged_attn_decode (plan_kernel + decode_tc_kernel)",
                      "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": dec_bytes,
                      "decode_ms": dec_ms},
         "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipelining": "uploads and downloads on two copy streams overlap the "
+                              "neighbouring steps' kernels (double-buffered device inputs)",
+                "pinned_h2d_gbs": h2d_gbs, "pinned_d2h_gbs": d2h_gbs,
+                "transfer_bound_ms": max(h2d / h2d_gbs, d2h / d2h_gbs) * 1e-6},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if contiguous:
         line["paged_vs_contiguous"] = contiguous
+    line.update(extras)
+    if "shared_prefix" in extras:
+        sp_x = extras["shared_prefix"]
+        sp_x["unique_gbs"] = sp_x["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, args.cpu_seconds)
     return line
