@@ -60,6 +60,9 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--contiguous", action="store_true",
                     help="also time the same batch with identity block placement")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="run kv_cache_append and paged_attn_decode as two calls instead of "
+                         "the fused paged_attn_decode_append")
     return ap.parse_args()
 
 
@@ -296,7 +299,7 @@ def config_block(case, workload, n_gpus):
         "partition_size": case.partition_size,
         "context_tokens_per_gpu": int(case.context_lens.sum()),
         "max_context_len": case.max_context_len,
-        "step": "kv_cache_append (newest token of each sequence) + paged_attn_decode",
+        "step": "append of each sequence's newest token + paged decode over its whole context",
         "accumulate": "fp32",
         "l2": "inputs larger than L2: the K/V pool read each step is "
               f"{case.k_pool.numel() * case.k_pool.element_size() * 2 / 1e9:.2f} GB per GPU",
@@ -394,24 +397,33 @@ def run_ours(args, rank, world, local_rank):
     ws_bytes = pkv.decode_workspace_bytes(S, Hq, D, mcl, case.partition_size)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    # append, then plan + decode (16-bit; the merge is fused into the decode),
-    # or decode + merge kernel when split (fp32)
+    # 16-bit: plan + decode (append and merge fused in), or append + plan +
+    # decode with --separate-append; fp32: append + decode (+ merge when split)
     if case.q.dtype == torch.float32:
         launches_per_step = 2 + (1 if mcl > case.partition_size > 0 else 0)
     else:
-        launches_per_step = 3
+        launches_per_step = 3 if args.separate_append else 2
 
     def decode(c, o):
         pkv.paged_attn_decode(o, c.q, c.k_pool, c.v_pool, c.block_tables, c.context_lens,
                               c.scale, mcl, partition_size=c.partition_size, workspace=ws,
                               err=err)
 
+    fused = not args.separate_append and case.q.dtype != torch.float32
+
     def step(ev_pair=None):
-        pkv.kv_cache_append(case.k_pool, case.v_pool, case.k_new, case.v_new,
-                            case.slot_mapping, err=err)
+        if not fused:
+            pkv.kv_cache_append(case.k_pool, case.v_pool, case.k_new, case.v_new,
+                                case.slot_mapping, err=err)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        decode(case, out)
+        if fused:
+            pkv.paged_attn_decode_append(out, case.q, case.k_new, case.v_new, case.k_pool,
+                                         case.v_pool, case.block_tables, case.context_lens,
+                                         case.scale, mcl, partition_size=case.partition_size,
+                                         workspace=ws, err=err)
+        else:
+            decode(case, out)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
@@ -462,7 +474,9 @@ def run_ours(args, rank, world, local_rank):
     # back, as a serving loop does. The copies run on two copy streams, with
     # double-buffered device inputs/outputs, so step i+1's upload and step
     # i-1's download overlap step i's kernels.
-    names = ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens")
+    names = ("q", "k_new", "v_new", "block_tables", "context_lens")
+    if not fused:
+        names = names + ("slot_mapping",)
     host_in = {k: getattr(case, k).cpu().pin_memory() for k in names}
     dev_sets = [{k: torch.empty_like(getattr(case, k)) for k in names} for _ in range(2)]
     outs = [torch.empty_like(out) for _ in range(2)]
@@ -476,6 +490,12 @@ def run_ours(args, rank, world, local_rank):
     out_free = [torch.cuda.Event() for _ in range(2)]
 
     def run_step(inp, o):
+        if fused:
+            pkv.paged_attn_decode_append(o, inp["q"], inp["k_new"], inp["v_new"], case.k_pool,
+                                         case.v_pool, inp["block_tables"], inp["context_lens"],
+                                         case.scale, mcl, partition_size=case.partition_size,
+                                         workspace=ws, err=err)
+            return
         pkv.kv_cache_append(case.k_pool, case.v_pool, inp["k_new"], inp["v_new"],
                             inp["slot_mapping"], err=err)
         pkv.paged_attn_decode(o, inp["q"], case.k_pool, case.v_pool, inp["block_tables"],
@@ -580,7 +600,7 @@ def run_ours(args, rank, world, local_rank):
         "seq_steps_per_s": S * world / (ms * 1e-3),
         "pct_of_hbm_peak": {"of_spec_8000_gbs": value / (HBM_SPEC_GBS * world),
                             f"of_{peak_kind}_{peak:.0f}_gbs": value / (peak * world)},
-        "roofline": {"kernel": "paged_attn_decode (plan_kernel + decode_tc_kernel)",
+        "roofline": {"kernel": "decode call (plan_kernel + decode_tc_kernel)",
                      "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": dec_bytes,
@@ -596,6 +616,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if contiguous:
         line["paged_vs_contiguous"] = contiguous
+    line["config"]["call"] = ("kv_cache_append + paged_attn_decode" if not fused else
+                              "paged_attn_decode_append (append fused into the decode)")
     line.update(extras)
     if "shared_prefix" in extras:
         sp_x = extras["shared_prefix"]

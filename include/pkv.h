@@ -167,6 +167,36 @@ int paged_attn_decode_static_ws(void *out, const void *q, const void *k_pool, co
                                 int32_t *err, void *stream);
 
 /*
+ * paged_attn_decode_append - one decode step with the cache-append fused in.
+ *
+ * For every sequence s with L = context_lens[s] >= 1 and every KV head h,
+ * token L-1 is the newest token: its K/V rows k_new[s][h][:] and
+ * v_new[s][h][:] are written into its pool slot (block
+ * block_tables[s][(L-1) / block_size], slot (L-1) % block_size). The decode is
+ * then paged_attn_decode over all L tokens, taking the newest one from
+ * k_new / v_new. The result equals kv_cache_append with
+ * slot_mapping[s] = block_tables[s][(L-1)/B]*B + (L-1)%B followed by
+ * paged_attn_decode, in one pass: the new rows travel with the sequence's
+ * work, so no separate append launch is needed. Page "PagedAttention Analysis"
+ * (ryotta.opik.net), section 3, notes that vLLM fuses its kernels to soften
+ * the cost of the block-table indirection.
+ *
+ * k_new, v_new  [num_seqs][num_kv_heads][head_dim], 16-byte aligned.
+ * k_pool, v_pool are written, at exactly those slots.
+ * Other arguments, errors and the workspace are those of paged_attn_decode.
+ * fp16 / bf16 only (PKV_EUNSUPPORTED for f32). Precondition: the last block
+ * of each sequence is its own. That holds after copy-on-write, which makes a
+ * shared block private before the first write into it.
+ */
+int paged_attn_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                             void *k_pool, void *v_pool, const int32_t *block_tables,
+                             const int32_t *context_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, int block_size,
+                             int max_blocks_per_seq, int num_blocks, int max_context_len,
+                             float scale, int dtype, int partition_size, void *workspace,
+                             size_t workspace_bytes, int32_t *err, void *stream);
+
+/*
  * kv_cache_append - write new tokens' K/V into their slots.
  *
  * For each token i < num_tokens with slot = slot_mapping[i] >= 0 and every KV

@@ -29,8 +29,8 @@ DEV_ERRORS = {1: "block id out of range", 2: "append slot out of range",
 DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DEFAULT_PARTITION = 2048  # tokens per split-context partition (measured best on B200)
 
-EXPORTS = ("paged_attn_decode", "kv_cache_append", "kv_block_copy",
-           "pkv_decode_workspace_bytes", "pkv_status_string")
+EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
+           "kv_block_copy", "pkv_decode_workspace_bytes", "pkv_status_string")
 
 
 class PkvError(RuntimeError):
@@ -55,6 +55,9 @@ def load_library():
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.paged_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, P, Z, P, P]
     lib.paged_attn_decode.restype = I
+    lib.paged_attn_decode_append.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F,
+                                             I, I, P, Z, P, P]
+    lib.paged_attn_decode_append.restype = I
     lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P]
     lib.kv_cache_append.restype = I
     lib.kv_block_copy.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
@@ -128,6 +131,46 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
         int(partition_size), _dev_ptr(workspace, "workspace", dev), ws_bytes,
         _dev_ptr(err, "err", dev), _stream_ptr(stream, dev))
     _check("paged_attn_decode", rc)
+    return out
+
+
+def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor,
+                             v_new: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                             block_tables: torch.Tensor, context_lens: torch.Tensor,
+                             scale: float, max_context_len: int,
+                             partition_size: int = DEFAULT_PARTITION,
+                             workspace: Optional[torch.Tensor] = None,
+                             err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step with the cache-append fused in: sequence s's newest token
+    (``k_new[s]``, ``v_new[s]``, [S][Hkv][D]) is written into the pool slot of its
+    token ``context_lens[s] - 1`` and attended over, in one pass (fp16/bf16)."""
+    lib = load_library()
+    dev = q.device
+    if q.dtype not in DTYPE_CODES or any(t.dtype != q.dtype
+                                         for t in (out, k_new, v_new, k_pool, v_pool)):
+        raise TypeError("q, out, k_new, v_new and the pools must share one dtype")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    S, Hq, D = (int(x) for x in q.shape)
+    P, Hkv, B, D2 = (int(x) for x in k_pool.shape)
+    if tuple(out.shape) != (S, Hq, D) or tuple(v_pool.shape) != (P, Hkv, B, D2) or D2 != D \
+            or tuple(k_new.shape) != (S, Hkv, D) or tuple(v_new.shape) != (S, Hkv, D):
+        raise ValueError("shape mismatch between q/out/k_new/v_new/pools")
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or tuple(context_lens.shape) != (S,):
+        raise ValueError("block_tables must be [S][max_blocks] and context_lens [S]")
+    need = decode_workspace_bytes(S, Hq, D, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.paged_attn_decode_append(
+        _dev_ptr(out, "out", dev), _dev_ptr(q, "q", dev), _dev_ptr(k_new, "k_new", dev),
+        _dev_ptr(v_new, "v_new", dev), _dev_ptr(k_pool, "k_pool", dev),
+        _dev_ptr(v_pool, "v_pool", dev), _dev_ptr(block_tables, "block_tables", dev),
+        _dev_ptr(context_lens, "context_lens", dev), S, Hq, Hkv, D, B,
+        int(block_tables.shape[1]), P, int(max_context_len), float(scale), DTYPE_CODES[q.dtype],
+        int(partition_size), _dev_ptr(workspace, "workspace", dev), ws_bytes,
+        _dev_ptr(err, "err", dev), _stream_ptr(stream, dev))
+    _check("paged_attn_decode_append", rc)
     return out
 
 

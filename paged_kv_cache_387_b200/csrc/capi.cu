@@ -114,12 +114,18 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int
   return pkv::workspace_layout(num_seqs, num_heads, head_dim, mp).total;
 }
 
-int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
-                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
-                      int num_heads, int num_kv_heads, int head_dim, int block_size,
-                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
-                      int dtype, int partition_size, void *workspace, size_t workspace_bytes,
-                      int32_t *err, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// paged_attn_decode, optionally with each sequence's newest token appended in
+// the same pass (k_new / v_new non-null; 16-bit only).
+int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool,
+                const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                int num_heads, int num_kv_heads, int head_dim, int block_size,
+                int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                int32_t *err, void *stream, const void *k_new, const void *v_new) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
       partition_size < 0)
@@ -189,6 +195,9 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
     a.ws_lse = reinterpret_cast<float *>(ws + wl.lse_off);
   }
 
+  a.k_new = k_new;
+  a.v_new = v_new;
+
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == PKV_F32) {
@@ -203,6 +212,38 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
   if (e != cudaSuccess) return PKV_ECUDA;
   if (mp > 1) return cuda_status(pkv::launch_merge(a, dtype, st));
   return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,
+                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                      int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
+                      int dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                      int32_t *err, void *stream) {
+  return decode_impl(out, q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                     num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                     max_context_len, scale, dtype, partition_size, workspace, workspace_bytes,
+                     err, stream, nullptr, nullptr);
+}
+
+int paged_attn_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                             void *k_pool, void *v_pool, const int32_t *block_tables,
+                             const int32_t *context_lens, int num_seqs, int num_heads,
+                             int num_kv_heads, int head_dim, int block_size,
+                             int max_blocks_per_seq, int num_blocks, int max_context_len,
+                             float scale, int dtype, int partition_size, void *workspace,
+                             size_t workspace_bytes, int32_t *err, void *stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return PKV_EINVAL;
+  if (num_seqs > 0 && (!aligned(k_new, 16) || !aligned(v_new, 16))) return PKV_EINVAL;
+  if (dtype == PKV_F32) return PKV_EUNSUPPORTED;
+  return decode_impl(out, q, k_pool, v_pool, block_tables, context_lens, num_seqs, num_heads,
+                     num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                     max_context_len, scale, dtype, partition_size, workspace, workspace_bytes,
+                     err, stream, k_new, v_new);
 }
 
 int kv_cache_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,

@@ -45,7 +45,8 @@
 //     rescaling rare. Masked tokens get -inf, and their V rows are zeroed in
 //     shared memory before they reach the tensor core.
 //   O^T[D][8] += V^T[D][16] . P^T[16][8]  V^T via ldmatrix.trans; P^T from the
-//     score fragment via movmatrix.trans (P rounded to the input type).
+//     score fragment via movmatrix.trans. P is split into hi + lo parts in the
+//     input type, two MMAs, so the weights keep ~16 significant bits.
 // At the end of an item the consumer warps' (max, sum, output) are combined in
 // shared memory. The result goes to `out` when the sequence has one
 // partition, and otherwise to the workspace as (normalised o_p,
@@ -77,7 +78,8 @@ constexpr int PLAN_BUCKETS = 64;     // size classes for ordering the short last
 
 // One entry of the scheduler -> consumer descriptor ring.
 struct ItemDesc {
-  int kind, s, p, h, L, n_tiles, nparts, pad;
+  int kind, s, p, h, L, n_tiles, nparts;
+  int new_tok;  // fused append: partition-relative index of token L-1, or -1
   int ids[DESC_TILES];  // physical block of tile t (tiles beyond: read from the table)
 };
 
@@ -91,11 +93,15 @@ struct TcShape {
   static constexpr int ACC_STRIDE = D + 4;               // padded combine row (floats)
   static constexpr int CW_FLOATS = NH * ACC_STRIDE + 2 * NH;  // acc[NH][D+4], m[NH], l[NH]
   static constexpr int COMBINE_BYTES = (NCW * CW_FLOATS + NH * (NCW + 1)) * 4;  // + scales
-  static constexpr int QBUF_BYTES = NH * D * 2;
+  // per slot: the group's q rows, then the newest token's K and V rows (fused append)
+  static constexpr int QROWS_BYTES = NH * D * 2;
+  static constexpr int QBUF_BYTES = QROWS_BYTES + 2 * D * 2;
   static constexpr int FIXED = COMBINE_BYTES + NSLOT * QBUF_BYTES +
                                NSLOT * (int)sizeof(ItemDesc) + 64 * 8 + 1024 + 64;
-  // As many stages as fit two CTAs per SM (about 110 KB each), at most 6.
-  static constexpr int NSTAGE_FIT = (110 * 1024 - FIXED) / (NCW * STAGE_BYTES);
+  // As many stages as fit two CTAs per SM, at most 6. An SM has 228 KB of
+  // shared memory and each CTA also reserves 1 KB, so a CTA may use ~113 KB.
+  static constexpr int CTA_SMEM_BUDGET = 228 * 1024 / 2 - 1024 - 256;
+  static constexpr int NSTAGE_FIT = (CTA_SMEM_BUDGET - FIXED) / (NCW * STAGE_BYTES);
   static constexpr int NSTAGE = NSTAGE_FIT > 6 ? 6 : NSTAGE_FIT;
   static_assert(NSTAGE >= 2, "ring too shallow");
   static constexpr int RING_BYTES = NCW * NSTAGE * STAGE_BYTES;
@@ -456,6 +462,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
       for (int t = lane; t < n_tiles && t < DESC_TILES; t += 32)
         d.ids[t] = bt[(t_begin + t * TILE) / B];
+      // Fused append: the partition holding token L-1 also stages that
+      // token's new K and V rows.
+      const bool has_new = a.k_new != nullptr && n_tiles > 0 && t_end == L;
       if (lane == 0) {
         d.kind = KIND_WORK;
         d.s = s;
@@ -464,15 +473,24 @@ __global__ void __launch_bounds__(THREADS, 2)
         d.L = L;
         d.n_tiles = n_tiles;
         d.nparts = (L + a.part_tokens - 1) / a.part_tokens;
+        d.new_tok = has_new ? L - 1 - t_begin : -1;
       }
       __syncwarp();  // every lane's ids precede lane 0's release below
       if (lane == 0) {
         const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
-        mbar_arrive_expect_tx(item_full(slot), qbytes);
+        const uint32_t rbytes = has_new ? (uint32_t)(D * 2) : 0u;
+        mbar_arrive_expect_tx(item_full(slot), qbytes + 2 * rbytes);
+        const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES;
         if (qbytes)
-          bulk_load(smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES,
-                    static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
+          bulk_load(stage, static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
                     item_full(slot));
+        if (rbytes) {
+          const size_t row = ((size_t)s * Hkv + h) * D;
+          bulk_load(stage + Shape::QROWS_BYTES, static_cast<const T *>(a.k_new) + row, rbytes,
+                    item_full(slot));
+          bulk_load(stage + Shape::QROWS_BYTES + D * 2, static_cast<const T *>(a.v_new) + row,
+                    rbytes, item_full(slot));
+        }
       }
       ++in_flight;
       item = __shfl_sync(FULL_MASK, next, 0);
@@ -590,6 +608,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     const int s = dref.s, p = dref.p, h = dref.h, L = dref.L, n_tiles = dref.n_tiles;
     const int nparts = dref.nparts;
+    const int new_tok = dref.new_tok;
     const int t_begin = p * a.part_tokens;
     const int nt_w = warp < n_tiles ? (n_tiles - warp + NCW - 1) / NCW : 0;
 
@@ -629,6 +648,30 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int valid = min(TILE, L - tok0);
       const bool bad = (bad_mask >> st) & 1u;
 
+      const int tile_idx = warp + j * NCW;
+      if (new_tok >= 0 && (new_tok >> 4) == tile_idx && !bad) {
+        // Fused append: this tile holds token L-1. Its K and V rows come from
+        // the staged new rows (whatever the pool slot held), and the same rows
+        // are written to the pool slot: that is the cache-append.
+        const int r = new_tok & (TILE - 1);
+        const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES +
+                               Shape::QROWS_BYTES;
+        constexpr int CH = D / 8;  // 16-byte chunks per row
+        const int e = lane % CH, kv = lane / CH;  // lanes 0..CH-1: K, CH..2CH-1: V
+        if (lane < 2 * CH) {
+          const uint4 v = lds128(stage + kv * D * 2 + e * 16);
+          const uint32_t tile_base = kv ? vs : ks;
+          sts128(tile_base + (e >> 3) * HALF_BYTES + r * 128 + (((e & 7) ^ (r & 7)) << 4), v);
+          const int tok = t_begin + new_tok;
+          const int phys = desc[slot].ids[tile_idx < DESC_TILES ? tile_idx : 0];
+          const int blk = tile_idx < DESC_TILES ? phys
+                                                : a.block_tables[(size_t)s * a.max_blocks + tok / B];
+          T *pool = static_cast<T *>(const_cast<void *>(kv ? a.v_pool : a.k_pool));
+          *reinterpret_cast<uint4 *>(pool + (((size_t)blk * Hkv + h) * B + tok % B) * D + e * 8) = v;
+        }
+        fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
+        __syncwarp();
+      }
       if (valid < TILE && !bad) {
         // Tokens past the context length: their V rows may hold anything
         // (NaN included); zero them so P*V stays finite.
@@ -694,8 +737,19 @@ __global__ void __launch_bounds__(THREADS, 2)
       l1 += p1 + p3;
 
       // P^T as the B operand: transpose the (token, head) fragment pairs.
-      const uint32_t pb0 = movmatrix_trans(pack2<T>(p0, p1));  // tokens 0..7
-      const uint32_t pb1 = movmatrix_trans(pack2<T>(p2, p3));  // tokens 8..15
+      // The tensor core takes P in the input type. P is carried as a sum of
+      // two such values (hi + lo). A single rounding, up to 2^-9 (bf16) or
+      // 2^-11 (fp16) per weight, can exceed the accuracy bound when value rows
+      // nearly cancel. The split brings P to about 16 (bf16) or 22 (fp16) bits.
+      const uint32_t w01 = pack2<T>(p0, p1), w23 = pack2<T>(p2, p3);
+      const uint32_t pb0 = movmatrix_trans(w01);  // tokens 0..7
+      const uint32_t pb1 = movmatrix_trans(w23);  // tokens 8..15
+      constexpr bool kSplitP = true;
+      uint32_t pl0 = 0, pl1 = 0;
+      if constexpr (kSplitP) {
+        pl0 = movmatrix_trans(pack2<T>(p0 - lo_half_to_float<T>(w01), p1 - hi_half_to_float<T>(w01)));
+        pl1 = movmatrix_trans(pack2<T>(p2 - lo_half_to_float<T>(w23), p3 - hi_half_to_float<T>(w23)));
+      }
 
       // ---- O^T += V^T . P^T ----
       const uint32_t vrow = vs + vr * 128;
@@ -706,6 +760,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         uint32_t r0, r1, r2, r3;
         ldsm_x4_trans(addr, r0, r1, r2, r3);
         mma16816<T>(acc[mt], r0, r1, r2, r3, pb0, pb1);
+        if constexpr (kSplitP) mma16816<T>(acc[mt], r0, r1, r2, r3, pl0, pl1);
       }
       __syncwarp();  // every lane is done with this stage before it is refilled
       ++done;

@@ -100,6 +100,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ void sts128_zero(uint32_t addr) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
 }
@@ -159,6 +165,28 @@ template <>
 __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// The float value of the low / high 16-bit half of a packed pair.
+template <typename T>
+__device__ __forceinline__ float lo_half_to_float(uint32_t w);
+template <typename T>
+__device__ __forceinline__ float hi_half_to_float(uint32_t w);
+template <>
+__device__ __forceinline__ float lo_half_to_float<__nv_bfloat16>(uint32_t w) {
+  return __uint_as_float(w << 16);
+}
+template <>
+__device__ __forceinline__ float hi_half_to_float<__nv_bfloat16>(uint32_t w) {
+  return __uint_as_float(w & 0xffff0000u);
+}
+template <>
+__device__ __forceinline__ float lo_half_to_float<__half>(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+}
+template <>
+__device__ __forceinline__ float hi_half_to_float<__half>(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
 // Hardware base-2 exponential (the PTX ex2.approx instruction; -inf -> +0).

@@ -29,6 +29,10 @@ struct DecodeArgs {
   int max_parts;       // partitions of the longest allowed context
   float scale_log2;    // scale * log2(e): scores are kept in base-2 units
   int32_t *err;        // nullable device error word
+  // Fused cache-append (or null): each sequence's newest token, [S][Hkv][D].
+  // The decode writes it into the pool slot of token L-1 and attends over it.
+  const void *k_new;
+  const void *v_new;
   // Work list of the persistent decode kernel (written by the plan kernel):
   uint32_t *work;      // [<= S*max_parts] (seq << 16 | partition), full partitions first
   int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries

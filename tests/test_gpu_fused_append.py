@@ -1,0 +1,83 @@
+"""paged_attn_decode_append (cache-append fused into decode) against the oracle:
+the pool after the call must equal the oracle's append bit for bit, and the
+output must match the oracle's decode over the appended cache."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_387_b200 as pkv
+from pkv_inputs import make_case, make_random_case, make_shared_prefix_case
+from tests.helpers import assert_close_to_oracle
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+DT = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def fused_vs_oracle(c, part, what):
+    kc, vc = c.k_pool.cpu(), c.v_pool.cpu()
+    oracle.cache_append(kc, vc, c.k_new.cpu(), c.v_new.cpu(), c.slot_mapping.cpu())
+    ref = oracle.paged_decode(c.q.cpu(), kc, vc, c.block_tables.cpu(), c.context_lens.cpu(),
+                              c.scale)
+    out = torch.empty_like(c.q)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attn_decode_append(out, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
+                                 c.block_tables, c.context_lens, c.scale, c.max_context_len,
+                                 partition_size=part, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(c.k_pool.cpu().view(torch.int16), kc.view(torch.int16)), what
+    assert torch.equal(c.v_pool.cpu().view(torch.int16), vc.view(torch.int16)), what
+    assert_close_to_oracle(out, ref, c.q.dtype, what)
+
+
+# every position of the newest token inside its tile and block, tile edges included
+LENS = [1, 2, 15, 16, 17, 31, 32, 33, 48, 100, 511, 512, 513, 1000, 2049]
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 64)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (8, 1)])
+@pytest.mark.parametrize("part", [0, 512, 2048])
+def test_fused_append_decode_matches_append_then_decode(dt, D, B, Hq, Hkv, part):
+    c = make_random_case("fused", Hq, Hkv, D, B, LENS, DT[dt], seed=D + B + Hq, device=DEV,
+                         with_append=True)
+    fused_vs_oracle(c, part, f"{dt} D{D} B{B} G{Hq // Hkv} p{part}")
+
+
+def test_fused_append_opt13b_workload():
+    c = make_case("opt13b_mha_b64", device=DEV)
+    fused_vs_oracle(c, c.partition_size, "opt13b fused")
+
+
+def test_fused_append_shared_prefix_pipeline():
+    sp = make_shared_prefix_case(device=DEV, decode_steps=20)
+    kc, vc = sp.k_pool.cpu(), sp.v_pool.cpu()
+    pkv.kv_block_copy(sp.k_pool, sp.v_pool, sp.cow_pairs)
+    oracle.block_copy(kc, vc, sp.cow_pairs.cpu())
+    for k, st in enumerate(sp.steps):
+        q, kn, vn = sp.step_tokens(k)
+        out = torch.empty_like(q)
+        pkv.paged_attn_decode_append(out, q, kn, vn, sp.k_pool, sp.v_pool, st["block_tables"],
+                                     st["context_lens"], sp.scale,
+                                     int(st["context_lens"].max()), partition_size=512)
+        oracle.cache_append(kc, vc, kn.cpu(), vn.cpu(), st["slot_mapping"].cpu())
+        if k in (0, 7, 19):
+            ref = oracle.paged_decode(q.cpu(), kc, vc, st["block_tables"].cpu(),
+                                      st["context_lens"].cpu(), sp.scale)
+            assert_close_to_oracle(out, ref, torch.float16, f"shared prefix fused step {k}")
+    torch.cuda.synchronize()
+    assert torch.equal(sp.k_pool.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(sp.v_pool.cpu().view(torch.int16), vc.view(torch.int16))
+
+
+def test_fused_append_rejects_fp32():
+    c = make_random_case("f32", 2, 2, 64, 16, [5], torch.float32, seed=1, device=DEV,
+                         with_append=True)
+    out = torch.empty_like(c.q)
+    with pytest.raises(pkv.PkvError) as e:
+        pkv.paged_attn_decode_append(out, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
+                                     c.block_tables, c.context_lens, c.scale, 5)
+    assert e.value.status == pkv.PKV_EUNSUPPORTED
