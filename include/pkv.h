@@ -67,7 +67,7 @@ enum {
 
 /*
  * Bytes of device workspace paged_attn_decode needs for these sizes: a few
- * scheduling words and the work list (one 4-byte entry per possible
+ * scheduling words and the work list (one 8-byte entry per possible
  * (sequence, partition) pair), plus, when a context can span several
  * partitions, one fp32 output row and one fp32 log-sum-exp per (sequence,
  * query head, partition). Always > 0 for num_seqs > 0. This function is pure

@@ -64,7 +64,7 @@ WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long lo
   w.sched_off = off;
   off += 256;
   w.work_off = off;
-  off += round_up((size_t)(S * max_parts) * sizeof(uint32_t), 256);
+  off += round_up((size_t)(S * max_parts) * sizeof(uint2), 256);
   if (max_parts > 1) {
     const long long chunks = (max_parts + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK;
     w.cnt_off = off;  // Hq >= Hkv bounds the (sequence, KV head) counters
@@ -182,7 +182,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
   if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 256)) return PKV_EINVAL;
   char *ws = static_cast<char *>(workspace);
   a.sched = reinterpret_cast<int32_t *>(ws + wl.sched_off);
-  a.work = reinterpret_cast<uint32_t *>(ws + wl.work_off);
+  a.work = reinterpret_cast<uint2 *>(ws + wl.work_off);
   a.max_chunks = (int)((mp + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK);
   if (mp > 1) {
     a.merge_cnt = reinterpret_cast<int32_t *>(ws + wl.cnt_off);

@@ -62,6 +62,11 @@ constexpr int TILE = 16;                 // tokens per tile (mma M for QK, K for
 constexpr int NCW = 4;                   // consumer warps
 constexpr int THREADS = (NCW + 1) * 32;  // + one scheduler warp
 constexpr int NSLOT = 3;                 // item descriptors in flight
+// Near the end of the work list a CTA holds at most two work descriptors (the
+// one being consumed and the next), so that the last items are spread over
+// the CTAs instead of queued in a few of them. "Near" = fewer than this many
+// items per CTA left.
+constexpr int END_ITEMS_PER_CTA = 6;
 constexpr int DESC_TILES = 64;           // tile block ids carried by a descriptor
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
@@ -118,12 +123,17 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
   return (static_cast<uint32_t>(s) << 16) | static_cast<uint32_t>(p);
 }
 
-// Build the work list: every sequence's full partitions first (all the same
-// size), then the shorter last partitions ordered by size, largest first
-// (a counting sort over PLAN_BUCKETS size classes). Handing out the largest
-// items first and the smallest last keeps the CTAs' finishing times close. A
-// sequence of length 0 gets one entry, so its output is still written. The
-// merge counters are reset here too.
+// Build the work list in two regions.
+//  1. Sequences that span several partitions: all their partitions, sequence
+//     by sequence, the short last partition first. Their merges then complete
+//     while the list is still being worked through.
+//  2. Sequences of one partition, ordered by size, largest first (a counting
+//     sort over PLAN_BUCKETS size classes). They need no merge, and handing out
+//     the largest first and the smallest last keeps the CTAs' finishing times
+//     close. A sequence of length 0 is one (empty) entry, so that its output is
+//     still written.
+// Each entry carries the sequence's clamped length. The merge counters are
+// reset here too.
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
   __shared__ int wsum[PLAN_THREADS / 32];
   __shared__ int hist[PLAN_BUCKETS];
@@ -140,22 +150,23 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   const int chunk = (S + PLAN_THREADS - 1) / PLAN_THREADS;
   const int s0 = min(S, tid * chunk), s1 = min(S, s0 + chunk);
   const int max_tiles = max(1, P / 16);
-  // size class of a last partition of `rem` tokens: bigger -> smaller bucket
-  auto bucket = [&](int rem) {
-    const int tiles = (rem + 15) / 16;
+  // size class of a one-partition sequence of `len` tokens: bigger -> smaller bucket
+  auto bucket = [&](int len) {
+    const int tiles = (len + 15) / 16;
     return (PLAN_BUCKETS - 1) - min(PLAN_BUCKETS - 1, tiles * (PLAN_BUCKETS - 1) / max_tiles);
   };
 
-  int nf = 0;
+  int nm = 0;  // region-1 entries of this thread's sequences
   for (int s = s0; s < s1; ++s) {
     const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
-                                a.block_size, nullptr);
-    nf += L / P;
-    const int rem = L % P;
-    if (rem != 0 || L == 0) atomicAdd(&hist[bucket(rem)], 1);
+                                a.block_size, a.err);
+    if (L > P)
+      nm += (L + P - 1) / P;
+    else
+      atomicAdd(&hist[bucket(L)], 1);
   }
-  // block-wide exclusive scan of the full-partition counts
-  int f = nf;
+  // block-wide exclusive scan of the region-1 counts
+  int f = nm;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int y = __shfl_up_sync(FULL_MASK, f, off);
@@ -173,9 +184,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     wsum[lane] = v;  // inclusive prefix over warps
   }
   __syncthreads();
-  const int base_f = (warp ? wsum[warp - 1] : 0) + f - nf;
-  const int total_f = wsum[PLAN_THREADS / 32 - 1];
-  // bucket offsets (exclusive scan of hist, after the full partitions)
+  const int base_m = (warp ? wsum[warp - 1] : 0) + f - nm;
+  const int total_m = wsum[PLAN_THREADS / 32 - 1];
+  // bucket offsets (exclusive scan of hist, after region 1)
   if (warp == 0) {
     const int h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
     int v = h0 + h1;
@@ -185,23 +196,26 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
       if (lane >= off) v += y;
     }
     const int excl = v - h0 - h1;
-    hist[2 * lane] = total_f + excl;
-    hist[2 * lane + 1] = total_f + excl + h0;
+    hist[2 * lane] = total_m + excl;
+    hist[2 * lane + 1] = total_m + excl + h0;
     if (lane == 31 && tid == 31) {
       a.sched[0] = 0;
-      a.sched[1] = total_f + v;
+      a.sched[1] = total_m + v;
     }
   }
   __syncthreads();
 
-  int of = base_f;
+  int om = base_m;
   for (int s = s0; s < s1; ++s) {
     const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
                                 a.block_size, nullptr);
-    const int full = L / P;
-    for (int q = 0; q < full; ++q) a.work[of++] = pack_pair(s, q);
-    const int rem = L % P;
-    if (rem != 0 || L == 0) a.work[atomicAdd(&hist[bucket(rem)], 1)] = pack_pair(s, full);
+    if (L > P) {
+      const int np = (L + P - 1) / P;
+      a.work[om++] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
+      for (int q = 0; q < np - 1; ++q) a.work[om++] = make_uint2(pack_pair(s, q), (uint32_t)L);
+    } else {
+      a.work[atomicAdd(&hist[bucket(L)], 1)] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+    }
   }
 }
 
@@ -378,10 +392,12 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ======================= scheduler warp =======================
     const long long list_cap = (long long)a.num_seqs * a.max_parts;
     const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
+    const int end_phase = total_items - END_ITEMS_PER_CTA * (int)gridDim.x;
     int item = 0;
     if (lane == 0) item = atomicAdd(&a.sched[0], 1);
     item = __shfl_sync(FULL_MASK, item, 0);
-    int in_flight = 0;  // posted work / merge descriptors whose completion is not yet handled
+    bool claimed = true;  // `item` holds an index taken from the work list
+    int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
     for (uint32_t it = 0;; ++it) {
       const int slot = it % NSLOT;
       ItemDesc &d = desc[slot];
@@ -436,6 +452,19 @@ __global__ void __launch_bounds__(THREADS, 2)
         ++in_flight;
         continue;
       }
+      if (!claimed) {
+        // End phase: claim the next item only once the descriptor posted two
+        // iterations ago is done, so at most two work descriptors are held.
+        if (it >= 2) {
+          const uint32_t o = it - 2;
+          if (!__all_sync(FULL_MASK, wait_or_abort(item_empty(o % NSLOT), (o / NSLOT) & 1,
+                                                   abort_flag, a.err)))
+            break;
+        }
+        if (lane == 0) item = atomicAdd(&a.sched[0], 1);
+        item = __shfl_sync(FULL_MASK, item, 0);
+        claimed = true;
+      }
       if (item >= total_items) {
         // No new work: keep the ring turning (no-op descriptors) until every
         // posted item has completed and produced its merge tasks, then stop.
@@ -447,15 +476,17 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (in_flight == 0) break;
         continue;
       }
+      // Before the end phase the next item is claimed now, so that its index
+      // is ready when this one has been posted.
+      const bool prefetch = item < end_phase;
       int next = 0;
-      if (lane == 0) next = atomicAdd(&a.sched[0], 1);  // consumed at the end of this item
+      if (prefetch && lane == 0) next = atomicAdd(&a.sched[0], 1);
 
-      const uint32_t pr = a.work[item / Hkv];
+      const uint2 wk = a.work[item / Hkv];
       const int h = item - (item / Hkv) * Hkv;
-      const int s = min(static_cast<int>(pr >> 16), a.num_seqs - 1);
-      const int p = static_cast<int>(pr & 0xffffu);
-      const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, B,
-                                  lane == 0 ? a.err : nullptr);
+      const int s = min(static_cast<int>(wk.x >> 16), a.num_seqs - 1);
+      const int p = static_cast<int>(wk.x & 0xffffu);
+      const int L = static_cast<int>(wk.y);  // clamped (and checked) by the plan
       const int t_begin = p * a.part_tokens;
       const int t_end = min(L, t_begin + a.part_tokens);
       const int n_tiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
@@ -493,7 +524,10 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
       }
       ++in_flight;
-      item = __shfl_sync(FULL_MASK, next, 0);
+      if (prefetch)
+        item = __shfl_sync(FULL_MASK, next, 0);
+      else
+        claimed = false;
     }
     return;
   }
@@ -737,14 +771,15 @@ __global__ void __launch_bounds__(THREADS, 2)
       l1 += p1 + p3;
 
       // P^T as the B operand: transpose the (token, head) fragment pairs.
-      // The tensor core takes P in the input type. P is carried as a sum of
-      // two such values (hi + lo). A single rounding, up to 2^-9 (bf16) or
-      // 2^-11 (fp16) per weight, can exceed the accuracy bound when value rows
-      // nearly cancel. The split brings P to about 16 (bf16) or 22 (fp16) bits.
+      // The tensor core takes P in the input type. One bf16 rounding (up to
+      // 2^-8 relative per weight) can exceed the accuracy bound when value
+      // rows nearly cancel, so for bf16 P is carried as hi + lo (about 16
+      // bits). For fp16 one rounding (2^-11) bounds the output error by
+      // 2^-11 * max|v|, inside the bound, and P stays a single operand.
       const uint32_t w01 = pack2<T>(p0, p1), w23 = pack2<T>(p2, p3);
       const uint32_t pb0 = movmatrix_trans(w01);  // tokens 0..7
       const uint32_t pb1 = movmatrix_trans(w23);  // tokens 8..15
-      constexpr bool kSplitP = true;
+      constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
       uint32_t pl0 = 0, pl1 = 0;
       if constexpr (kSplitP) {
         pl0 = movmatrix_trans(pack2<T>(p0 - lo_half_to_float<T>(w01), p1 - hi_half_to_float<T>(w01)));

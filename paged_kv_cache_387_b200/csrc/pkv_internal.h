@@ -34,7 +34,7 @@ struct DecodeArgs {
   const void *k_new;
   const void *v_new;
   // Work list of the persistent decode kernel (written by the plan kernel):
-  uint32_t *work;      // [<= S*max_parts] (seq << 16 | partition), full partitions first
+  uint2 *work;         // [<= S*max_parts] {seq << 16 | partition, context length}, fulls first
   int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries
   // Partition merging (split contexts). Partitions are merged in chunks of
   // MERGE_CHUNK; a context with more than one chunk is merged in two levels.

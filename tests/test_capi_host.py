@@ -53,14 +53,14 @@ def test_status_strings(lib):
 
 def test_workspace_arithmetic(lib):
     f = lib.pkv_decode_workspace_bytes
-    # scheduling words (256 B) + work list (one uint32 per (seq, partition)),
+    # scheduling words (256 B) + work list (8 bytes per (seq, partition)),
     # each region rounded up to 256 B
     assert f(8, 32, 128, 512, 512) == 256 + 256   # one partition: no partials
     assert f(8, 32, 128, 100, 0) == 256 + 256     # unsplit
     # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16): chunk and
     # final merge counters, fp32 partition outputs + lse, chunk results + lse
     S, Hq, D, P, C = 8, 32, 128, 256, 16
-    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 4 + S * Hq * C * 4 + S * Hq * 4
+    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + S * Hq * C * 4 + S * Hq * 4
                                         + S * Hq * P * D * 4 + S * Hq * P * 4
                                         + S * Hq * C * D * 4 + S * Hq * C * 4)
     # 33 tokens in 16-token partitions = 3 partitions, one merge chunk
