@@ -70,7 +70,7 @@ constexpr int END_ITEMS_PER_CTA = 6;
 constexpr int DESC_TILES = 64;           // tile block ids carried by a descriptor
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
-constexpr int PLAN_THREADS = 1024;
+constexpr int PLAN_THREADS = 256;
 constexpr float RESCALE_SLACK = 8.f;     // lazy max: rescale only past 2^8 growth
 
 // Descriptor kinds (in ItemDesc::kind).
@@ -135,9 +135,13 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
 // Each entry carries the sequence's clamped length. The merge counters are
 // reset here too.
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
-  __shared__ int wsum[PLAN_THREADS / 32];
+  constexpr int NW = PLAN_THREADS / 32;
+  __shared__ int wsum[NW];
   __shared__ int hist[PLAN_BUCKETS];
   pdl_launch_dependents();  // the decode grid may launch; it waits for this grid to finish
+  // This grid may itself start while the previous decode call is finishing:
+  // nothing in global memory is touched before that call has completed.
+  pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, P = a.part_tokens;
   if (a.merge_cnt) {
@@ -175,17 +179,17 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   if (lane == 31) wsum[warp] = f;
   __syncthreads();
   if (warp == 0) {
-    int v = wsum[lane];
+    int v = lane < NW ? wsum[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(FULL_MASK, v, off);
       if (lane >= off) v += y;
     }
-    wsum[lane] = v;  // inclusive prefix over warps
+    if (lane < NW) wsum[lane] = v;  // inclusive prefix over warps
   }
   __syncthreads();
   const int base_m = (warp ? wsum[warp - 1] : 0) + f - nm;
-  const int total_m = wsum[PLAN_THREADS / 32 - 1];
+  const int total_m = wsum[NW - 1];
   // bucket offsets (exclusive scan of hist, after region 1)
   if (warp == 0) {
     const int h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     hist[2 * lane] = total_m + excl;
     hist[2 * lane + 1] = total_m + excl + h0;
     if (lane == 31 && tid == 31) {
-      a.sched[0] = 0;
+      a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
       a.sched[1] = total_m + v;
     }
   }
@@ -379,6 +383,9 @@ __global__ void __launch_bounds__(THREADS, 2)
     fence_mbar_init();
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
+  }
+  pdl_wait();  // the work list, counters and everything before the plan are ready
+  if (threadIdx.x == 0) {
     // A CTA that starts after some wait already gave up does no work.
     s_abort = (a.err != nullptr &&
                *reinterpret_cast<volatile const int32_t *>(a.err) == PKV_DEV_WAIT_TIMEOUT)
@@ -386,16 +393,13 @@ __global__ void __launch_bounds__(THREADS, 2)
                   : 0;
   }
   __syncthreads();
-  pdl_wait();  // the work list, counters and everything before the plan are ready
 
   if (warp == NCW) {
     // ======================= scheduler warp =======================
     const long long list_cap = (long long)a.num_seqs * a.max_parts;
     const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
     const int end_phase = total_items - END_ITEMS_PER_CTA * (int)gridDim.x;
-    int item = 0;
-    if (lane == 0) item = atomicAdd(&a.sched[0], 1);
-    item = __shfl_sync(FULL_MASK, item, 0);
+    int item = blockIdx.x;  // the first item of every CTA is fixed; the counter starts at grid
     bool claimed = true;  // `item` holds an index taken from the work list
     int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
     for (uint32_t it = 0;; ++it) {
@@ -529,6 +533,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       else
         claimed = false;
     }
+    // This CTA posts nothing more: the next call's grids may start launching
+    // (they wait for this grid to complete before touching memory).
+    if (lane == 0) pdl_launch_dependents();
     return;
   }
 
@@ -902,24 +909,34 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   long long grid = (long long)sm_count_for_current_device() * per_sm;
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
+  DecodeArgs b = a;
+  b.grid = (int)grid;
 
-  plan_kernel<<<1, PLAN_THREADS, 0, stream>>>(a);
-  e = cudaGetLastError();
+  // Both launches are programmatic dependents of what precedes them in the
+  // stream. The plan may start while a previous decode call finishes (it
+  // waits for that call before touching memory); the decode CTAs start
+  // (barrier set-up, descriptor prefetch) while the plan runs, and wait for
+  // it before reading the work list.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t pcfg = {};
+  pcfg.gridDim = dim3(1);
+  pcfg.blockDim = dim3(PLAN_THREADS);
+  pcfg.dynamicSmemBytes = 0;
+  pcfg.stream = stream;
+  pcfg.attrs = attr;
+  pcfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&pcfg, plan_kernel, b);
   if (e != cudaSuccess) return e;
-  // Programmatic dependent launch: the decode CTAs start (barrier set-up,
-  // descriptor prefetch) while the plan runs, and wait for it before reading
-  // the work list.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, a);
+  return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, b);
 }
 
 template <typename T>

@@ -43,6 +43,7 @@ struct DecodeArgs {
   float *ws2_o;        // [S][Hq][max_chunks][D] chunk results (normalised), or null
   float *ws2_lse;      // [S][Hq][max_chunks] chunk log2-sum-exp, or null
   int max_chunks;      // ceil(max_parts / MERGE_CHUNK)
+  int grid;            // CTAs of the decode grid (each takes item blockIdx.x first)
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
