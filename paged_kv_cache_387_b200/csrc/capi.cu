@@ -39,15 +39,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
 // A pool viewed as a 2-D tensor [rows = num_blocks*Hkv*B][D] of 16-bit
 // elements. It is read in boxes of 64 elements x 16 rows under the 128-byte
 // swizzle.
+// The pool as rows of head_dim 16-bit elements. A 128-byte swizzled box row
+// holds 64 elements, so a row of head_dim = 128 is two 64-element halves. For
+// that case the map is 3D, {64 elements, rows, halves}, with the halves
+// 128 bytes apart: one box {64, 16, 2} then lands as [half][16 rows][128 B],
+// a whole 16-token tile in one copy. head_dim = 64 uses the 2D map {64, rows}.
 bool make_pool_map(CUtensorMap *map, const void *pool, long long rows, int head_dim) {
   auto fn = encode_tiled_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  cuuint32_t box[2] = {64, 16};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(pool), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const int halves = head_dim / 64;
+  cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)halves};
+  cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, 128};
+  cuuint32_t box[3] = {64, 16, (cuuint32_t)halves};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, halves > 1 ? 3 : 2,
+                  const_cast<void *>(pool), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

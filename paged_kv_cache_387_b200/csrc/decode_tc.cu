@@ -611,10 +611,12 @@ __global__ void __launch_bounds__(THREADS, 2)
         const uint32_t kdst = ring + st * Shape::STAGE_BYTES;
         const uint32_t vdst = kdst + Shape::KT_BYTES;
         mbar_arrive_expect_tx(bar, Shape::STAGE_BYTES);
-#pragma unroll
-        for (int hh = 0; hh < Shape::HALVES; ++hh) {
-          tma_load_2d(kdst + hh * HALF_BYTES, &tmK, hh * BOX_COLS, y, bar);
-          tma_load_2d(vdst + hh * HALF_BYTES, &tmV, hh * BOX_COLS, y, bar);
+        if constexpr (Shape::HALVES == 1) {
+          tma_load_2d(kdst, &tmK, 0, y, bar);
+          tma_load_2d(vdst, &tmV, 0, y, bar);
+        } else {  // both halves of the tile in one copy each (3D map)
+          tma_load_3d(kdst, &tmK, 0, y, 0, bar);
+          tma_load_3d(vdst, &tmV, 0, y, 0, bar);
         }
       }
       ++issued;
