@@ -11,8 +11,13 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * Pointers. Every data pointer is a DEVICE pointer owned by the caller. The
- * library never allocates, frees or retains memory. Block allocation is host
+ * Pointers. Every data pointer is a DEVICE pointer owned by the caller, with
+ * one exception: the `out` of the decode entry points may also be page-locked
+ * host memory that the device addresses directly (unified addressing, e.g.
+ * from cudaHostAlloc). The kernels then write the result over the bus with
+ * plain stores, and no separate device-to-host copy is needed; the caller
+ * reads it once the stream has passed the call. The library never allocates,
+ * frees or retains memory. Block allocation is host
  * bookkeeping over integer block ids, and needs no device allocation during
  * generation (page "추론 엔진에서의 메모리 가상화", molayo1419.me, block
  * manager section).
@@ -97,7 +102,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
  * log-sum-exp weights.
  *
  * out            [num_seqs][num_heads][head_dim], written entirely. A sequence
- *                with L <= 0 gets zeros.
+ *                with L <= 0 gets zeros. Device memory, or page-locked host
+ *                memory the device can address (see Pointers).
  * q              [num_seqs][num_heads][head_dim]
  * k_pool, v_pool [num_blocks][num_kv_heads][block_size][head_dim]. Must be
  *                16-byte aligned.

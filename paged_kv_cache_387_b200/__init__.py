@@ -88,6 +88,18 @@ def _dev_ptr(t: Optional[torch.Tensor], name: str, device=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _out_ptr(t: torch.Tensor, device):
+    """`out` of a decode call: a CUDA tensor on `device`, or a page-locked
+    (pinned) host tensor, which the kernels write directly over the bus."""
+    if isinstance(t, torch.Tensor) and t.device.type == "cpu":
+        if not t.is_pinned():
+            raise ValueError("out on the host must be pinned (page-locked) memory")
+        if not t.is_contiguous():
+            raise ValueError("out must be contiguous")
+        return ctypes.c_void_p(t.data_ptr())
+    return _dev_ptr(t, "out", device)
+
+
 def _stream_ptr(stream, device):
     s = torch.cuda.current_stream(device) if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -124,7 +136,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     rc = lib.paged_attn_decode(
-        _dev_ptr(out, "out", dev), _dev_ptr(q, "q", dev), _dev_ptr(k_pool, "k_pool", dev),
+        _out_ptr(out, dev), _dev_ptr(q, "q", dev), _dev_ptr(k_pool, "k_pool", dev),
         _dev_ptr(v_pool, "v_pool", dev), _dev_ptr(block_tables, "block_tables", dev),
         _dev_ptr(context_lens, "context_lens", dev), S, Hq, Hkv, D, B,
         int(block_tables.shape[1]), P, int(max_context_len), float(scale), DTYPE_CODES[q.dtype],
@@ -163,7 +175,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     rc = lib.paged_attn_decode_append(
-        _dev_ptr(out, "out", dev), _dev_ptr(q, "q", dev), _dev_ptr(k_new, "k_new", dev),
+        _out_ptr(out, dev), _dev_ptr(q, "q", dev), _dev_ptr(k_new, "k_new", dev),
         _dev_ptr(v_new, "v_new", dev), _dev_ptr(k_pool, "k_pool", dev),
         _dev_ptr(v_pool, "v_pool", dev), _dev_ptr(block_tables, "block_tables", dev),
         _dev_ptr(context_lens, "context_lens", dev), S, Hq, Hkv, D, B,

@@ -111,3 +111,13 @@ def test_binding_refuses_cpu_tensors(lib):
     bt = torch.zeros(2, 1, dtype=torch.int32)
     with pytest.raises(ValueError):
         pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
+
+
+def test_binding_refuses_unpinned_host_output(lib):
+    """A host `out` is accepted only when it is page-locked."""
+    import torch
+    x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="pinned"):
+        pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)

@@ -81,3 +81,28 @@ def test_fused_append_rejects_fp32():
         pkv.paged_attn_decode_append(out, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
                                      c.block_tables, c.context_lens, c.scale, 5)
     assert e.value.status == pkv.PKV_EUNSUPPORTED
+
+
+@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("part", [0, 512])
+def test_output_into_pinned_host_memory(fused, part):
+    """`out` may be page-locked host memory: the kernels write it over the bus,
+    bit for bit what they write into device memory (merged partitions included)."""
+    c = make_random_case("pinned_out", 16, 4, 128, 16, LENS, torch.bfloat16, seed=7, device=DEV,
+                         with_append=True)
+    if not fused:
+        pkv.kv_cache_append(c.k_pool, c.v_pool, c.k_new, c.v_new, c.slot_mapping)
+    dev_out = torch.empty_like(c.q)
+    host_out = torch.full(tuple(c.q.shape), float("nan"), dtype=c.q.dtype).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for o in (dev_out, host_out):
+        if fused:  # appending the same token twice leaves the pool unchanged
+            pkv.paged_attn_decode_append(o, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
+                                         c.block_tables, c.context_lens, c.scale,
+                                         c.max_context_len, partition_size=part, err=err)
+        else:
+            pkv.paged_attn_decode(o, c.q, c.k_pool, c.v_pool, c.block_tables, c.context_lens,
+                                  c.scale, c.max_context_len, partition_size=part, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(dev_out.cpu().view(torch.int16), host_out.view(torch.int16))
