@@ -122,7 +122,9 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
  * err            nullable device int32 error word (see above).
  *
  * Supported: head_dim in {64, 128}; f32 with any block_size >= 1; f16/bf16
- * with block_size a multiple of 16 (up to 256) and num_heads/num_kv_heads <= 8.
+ * with block_size a multiple of 8 (up to 256) and num_heads/num_kv_heads <= 8.
+ * A block id outside [0, num_blocks) masks the tokens of its 16-token tile
+ * (with block_size 8 or another odd multiple of 8, a tile spans two blocks).
  * Anything else returns PKV_EUNSUPPORTED.
  */
 int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *v_pool,

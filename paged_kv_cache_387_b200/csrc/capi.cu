@@ -44,18 +44,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
 // that case the map is 3D, {64 elements, rows, halves}, with the halves
 // 128 bytes apart: one box {64, 16, 2} then lands as [half][16 rows][128 B],
 // a whole 16-token tile in one copy. head_dim = 64 uses the 2D map {64, rows}.
-bool make_pool_map(CUtensorMap *map, const void *pool, long long rows, int head_dim) {
+bool make_pool_map(CUtensorMap *map, const void *pool, long long rows, int head_dim,
+                   bool unit8) {
   auto fn = encode_tiled_fn();
   if (!fn) return false;
+  CUresult r;
+  if (unit8) {
+    // Block sizes that are odd multiples of 8: one box is 8 rows of one
+    // 64-element half (2D map), so each 8-token unit of a tile is fetched
+    // from its own block.
+    cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+    cuuint32_t box[2] = {64, 8};
+    cuuint32_t estr[2] = {1, 1};
+    r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void *>(pool), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+  }
   const int halves = head_dim / 64;
   cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)halves};
   cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, 128};
   cuuint32_t box[3] = {64, 16, (cuuint32_t)halves};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, halves > 1 ? 3 : 2,
-                  const_cast<void *>(pool), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, halves > 1 ? 3 : 2, const_cast<void *>(pool), dims,
+         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -153,7 +167,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
 
   long long rows = 0;  // pool rows of the TMA view (16-bit path)
   if (dtype != PKV_F32) {
-    if (block_size % 16 != 0 || block_size > 256) return PKV_EUNSUPPORTED;
+    if (block_size % 8 != 0 || block_size > 256) return PKV_EUNSUPPORTED;
     if (num_heads / num_kv_heads > 8) return PKV_EUNSUPPORTED;
     rows = (long long)num_blocks * num_kv_heads * block_size;
     if (rows > 0x7fffffffLL - 64) return PKV_EUNSUPPORTED;
@@ -172,6 +186,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
   a.num_kv_heads = num_kv_heads;
   a.head_dim = head_dim;
   a.block_size = block_size;
+  a.unit8 = block_size % 16 != 0 ? 1 : 0;
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
   a.max_context_len = max_context_len;
@@ -211,7 +226,8 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
     e = pkv::launch_decode_simt_f32(a, st);
   } else {
     CUtensorMap tmK, tmV;
-    if (!make_pool_map(&tmK, k_pool, rows, head_dim) || !make_pool_map(&tmV, v_pool, rows, head_dim))
+    if (!make_pool_map(&tmK, k_pool, rows, head_dim, a.unit8 != 0) ||
+        !make_pool_map(&tmV, v_pool, rows, head_dim, a.unit8 != 0))
       return PKV_ECUDA;
     // plan + decode; the partition merge is fused into the decode kernel
     return cuda_status(pkv::launch_decode_tc(a, dtype, tmK, tmV, st));

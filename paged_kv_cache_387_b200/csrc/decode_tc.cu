@@ -67,7 +67,10 @@ constexpr int NSLOT = 3;                 // item descriptors in flight
 // the CTAs instead of queued in a few of them. "Near" = fewer than this many
 // items per CTA left.
 constexpr int END_ITEMS_PER_CTA = 6;
-constexpr int DESC_TILES = 64;           // tile block ids carried by a descriptor
+// Block ids a descriptor carries: one per 16-token tile, or one per 8-token
+// unit when the block size is an odd multiple of 8. Further ids are read
+// from the table when their tile is fetched.
+constexpr int DESC_IDS = 64;
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
 constexpr int PLAN_THREADS = 256;
@@ -85,7 +88,7 @@ constexpr int PLAN_BUCKETS = 64;     // size classes for ordering the short last
 struct ItemDesc {
   int kind, s, p, h, L, n_tiles, nparts;
   int new_tok;  // fused append: partition-relative index of token L-1, or -1
-  int ids[DESC_TILES];  // physical block of tile t (tiles beyond: read from the table)
+  int ids[DESC_IDS];    // physical block of tile (or 8-token unit) t; -1 past the context
 };
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base). NH is
@@ -347,7 +350,9 @@ __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int 
   }
 }
 
-template <typename T, int D, int NH>
+// U8: the block size is an odd multiple of 8, so a 16-token tile is two
+// 8-token units that may sit in different blocks.
+template <typename T, int D, int NH, bool U8>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
@@ -495,8 +500,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int t_end = min(L, t_begin + a.part_tokens);
       const int n_tiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
       const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
-      for (int t = lane; t < n_tiles && t < DESC_TILES; t += 32)
-        d.ids[t] = bt[(t_begin + t * TILE) / B];
+      constexpr int upt = U8 ? 2 : 1;  // table entries per tile
+      for (int t = lane; t < n_tiles * upt && t < DESC_IDS; t += 32) {
+        const int tok = t_begin + t * (TILE / upt);
+        d.ids[t] = tok < L ? bt[tok / B] : -1;  // no table entry is read past the context
+      }
       // Fused append: the partition holding token L-1 also stages that
       // token's new K and V rows.
       const bool has_new = a.k_new != nullptr && n_tiles > 0 && t_end == L;
@@ -558,7 +566,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint32_t issued = 0, done = 0;  // tiles of this warp issued / consumed so far
   uint32_t bad_mask = 0;          // bit st: the tile in stage st had an invalid block id
   uint32_t is_it = 0;             // descriptor being issued
-  int is_j = 0, is_ntw = 0, is_h = 0, is_tbegin = 0, is_s = 0;
+  int is_j = 0, is_ntw = 0, is_h = 0, is_tbegin = 0, is_s = 0, is_L = 0;
   bool is_ready = false, is_end = false;
 
   // Issue this warp's next tiles while fewer than NSTAGE are in flight. With
@@ -581,6 +589,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
         const int nt = d.kind == KIND_WORK ? d.n_tiles : 0;
         is_s = d.s;
+        is_L = d.L;
         is_h = d.h;
         is_tbegin = d.p * a.part_tokens;
         is_ntw = warp < nt ? (nt - warp + NCW - 1) / NCW : 0;
@@ -594,29 +603,50 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       const int tile = warp + is_j * NCW;
       const int tok0 = is_tbegin + tile * TILE;
-      const int phys = tile < DESC_TILES ? desc[is_it % NSLOT].ids[tile]
-                                         : a.block_tables[(size_t)is_s * a.max_blocks + tok0 / B];
       const int st = issued % NSTAGE;
-      const bool bad = phys < 0 || phys >= a.num_blocks;
+      // Pool row of each unit of the tile. total_rows is wholly out of
+      // bounds, and TMA fills zeros there. It is used for an invalid block id,
+      // which is reported, and for a second unit past the context, whose
+      // table entry is not read. The first unit always starts before L.
+      constexpr int upt = U8 ? 2 : 1;
+      const int idx0 = tile * upt;
+      const int p0 = idx0 < DESC_IDS ? desc[is_it % NSLOT].ids[idx0]
+                                     : a.block_tables[(size_t)is_s * a.max_blocks + tok0 / B];
+      bool bad = p0 < 0 || p0 >= a.num_blocks;
+      const int y0 = bad ? total_rows : (p0 * Hkv + is_h) * B + (tok0 % B);
+      int y1 = total_rows;
+      if (U8 && tok0 + TILE / 2 < is_L) {
+        const int tok1 = tok0 + TILE / 2;
+        const int p1 = idx0 + 1 < DESC_IDS
+                           ? desc[is_it % NSLOT].ids[idx0 + 1]
+                           : a.block_tables[(size_t)is_s * a.max_blocks + tok1 / B];
+        const bool bad1 = p1 < 0 || p1 >= a.num_blocks;
+        bad = bad || bad1;
+        if (!bad1) y1 = (p1 * Hkv + is_h) * B + (tok1 % B);
+      }
       bad_mask = bad ? (bad_mask | (1u << st)) : (bad_mask & ~(1u << st));
       if (lane == 0) {
-        int y;
-        if (bad) {
-          report(a.err, PKV_DEV_BAD_BLOCK);
-          y = total_rows;  // wholly out of bounds: TMA fills zeros
-        } else {
-          y = (phys * Hkv + is_h) * B + (tok0 % B);
-        }
+        if (bad) report(a.err, PKV_DEV_BAD_BLOCK);
         const uint32_t bar = tile_full(warp, st);
         const uint32_t kdst = ring + st * Shape::STAGE_BYTES;
         const uint32_t vdst = kdst + Shape::KT_BYTES;
         mbar_arrive_expect_tx(bar, Shape::STAGE_BYTES);
-        if constexpr (Shape::HALVES == 1) {
-          tma_load_2d(kdst, &tmK, 0, y, bar);
-          tma_load_2d(vdst, &tmV, 0, y, bar);
+        if constexpr (U8) {
+          // two 8-row boxes per 64-element half (2D map): rows 0-7 and 8-15
+#pragma unroll
+          for (int hh = 0; hh < Shape::HALVES; ++hh) {
+            const uint32_t o = hh * HALF_BYTES;
+            tma_load_2d(kdst + o, &tmK, hh * BOX_COLS, y0, bar);
+            tma_load_2d(kdst + o + HALF_BYTES / 2, &tmK, hh * BOX_COLS, y1, bar);
+            tma_load_2d(vdst + o, &tmV, hh * BOX_COLS, y0, bar);
+            tma_load_2d(vdst + o + HALF_BYTES / 2, &tmV, hh * BOX_COLS, y1, bar);
+          }
+        } else if constexpr (Shape::HALVES == 1) {
+          tma_load_2d(kdst, &tmK, 0, y0, bar);
+          tma_load_2d(vdst, &tmV, 0, y0, bar);
         } else {  // both halves of the tile in one copy each (3D map)
-          tma_load_3d(kdst, &tmK, 0, y, 0, bar);
-          tma_load_3d(vdst, &tmV, 0, y, 0, bar);
+          tma_load_3d(kdst, &tmK, 0, y0, 0, bar);
+          tma_load_3d(vdst, &tmV, 0, y0, 0, bar);
         }
       }
       ++issued;
@@ -706,9 +736,9 @@ __global__ void __launch_bounds__(THREADS, 2)
           const uint32_t tile_base = kv ? vs : ks;
           sts128(tile_base + (e >> 3) * HALF_BYTES + r * 128 + (((e & 7) ^ (r & 7)) << 4), v);
           const int tok = t_begin + new_tok;
-          const int phys = desc[slot].ids[tile_idx < DESC_TILES ? tile_idx : 0];
-          const int blk = tile_idx < DESC_TILES ? phys
-                                                : a.block_tables[(size_t)s * a.max_blocks + tok / B];
+          const int idx = U8 ? tile_idx * 2 + (r >> 3) : tile_idx;
+          const int blk = idx < DESC_IDS ? desc[slot].ids[idx]
+                                         : a.block_tables[(size_t)s * a.max_blocks + tok / B];
           T *pool = static_cast<T *>(const_cast<void *>(kv ? a.v_pool : a.k_pool));
           *reinterpret_cast<uint4 *>(pool + (((size_t)blk * Hkv + h) * B + tok % B) * D + e * 8) = v;
         }
@@ -895,11 +925,11 @@ int sm_count_for_current_device() {
   return n;
 }
 
-template <typename T, int D, int NH>
+template <typename T, int D, int NH, bool U8>
 cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                       cudaStream_t stream) {
   using Shape = TcShape<D, NH>;
-  auto kern = decode_tc_kernel<T, D, NH>;
+  auto kern = decode_tc_kernel<T, D, NH, U8>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Shape::SMEM_BYTES);
   if (e != cudaSuccess) return e;
@@ -941,15 +971,15 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, b);
 }
 
-template <typename T>
+template <typename T, bool U8>
 cudaError_t launch_tc_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                         cudaStream_t stream) {
   const int G = a.num_heads / a.num_kv_heads;
   if (a.head_dim == 64)
-    return G <= 4 ? launch_tc<T, 64, 4>(a, tmK, tmV, stream)
-                  : launch_tc<T, 64, 8>(a, tmK, tmV, stream);
-  return G <= 4 ? launch_tc<T, 128, 4>(a, tmK, tmV, stream)
-                : launch_tc<T, 128, 8>(a, tmK, tmV, stream);
+    return G <= 4 ? launch_tc<T, 64, 4, U8>(a, tmK, tmV, stream)
+                  : launch_tc<T, 64, 8, U8>(a, tmK, tmV, stream);
+  return G <= 4 ? launch_tc<T, 128, 4, U8>(a, tmK, tmV, stream)
+                : launch_tc<T, 128, 8, U8>(a, tmK, tmV, stream);
 }
 
 }  // namespace
@@ -960,8 +990,11 @@ size_t decode_tc_smem_bytes(int head_dim) {
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t stream) {
-  if (dtype == PKV_BF16) return launch_tc_t<__nv_bfloat16>(a, tmK, tmV, stream);
-  return launch_tc_t<__half>(a, tmK, tmV, stream);
+  if (dtype == PKV_BF16)
+    return a.unit8 ? launch_tc_t<__nv_bfloat16, true>(a, tmK, tmV, stream)
+                   : launch_tc_t<__nv_bfloat16, false>(a, tmK, tmV, stream);
+  return a.unit8 ? launch_tc_t<__half, true>(a, tmK, tmV, stream)
+                 : launch_tc_t<__half, false>(a, tmK, tmV, stream);
 }
 
 }  // namespace pkv

@@ -44,6 +44,8 @@ struct DecodeArgs {
   float *ws2_lse;      // [S][Hq][max_chunks] chunk log2-sum-exp, or null
   int max_chunks;      // ceil(max_parts / MERGE_CHUNK)
   int grid;            // CTAs of the decode grid (each takes item blockIdx.x first)
+  int unit8;           // 1 when block_size % 16 == 8: a 16-token tile is two 8-token units
+                       // that may sit in different blocks
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level

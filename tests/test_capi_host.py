@@ -87,7 +87,8 @@ def test_decode_argument_checks(lib):
     assert decode(lib, scale=float("nan")) == pkv.PKV_EINVAL
     assert decode(lib, L=2048, ws=None, wsb=0) == pkv.PKV_EINVAL     # workspace needed
     assert decode(lib, D=96) == pkv.PKV_EUNSUPPORTED
-    assert decode(lib, B=8) == pkv.PKV_EUNSUPPORTED                   # 16-bit needs B % 16 == 0
+    assert decode(lib, B=12) == pkv.PKV_EUNSUPPORTED                  # 16-bit needs B % 8 == 0
+    assert decode(lib, B=264) == pkv.PKV_EUNSUPPORTED                 # and B <= 256
     assert decode(lib, Hq=32, Hkv=2) == pkv.PKV_EUNSUPPORTED          # group of 16 > 8
     assert decode(lib, q=ctypes.c_void_p(0x10008)) == pkv.PKV_EINVAL  # misaligned
     assert decode(lib, S=0) == pkv.PKV_OK                             # nothing to do

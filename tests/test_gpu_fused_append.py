@@ -38,7 +38,7 @@ LENS = [1, 2, 15, 16, 17, 31, 32, 33, 48, 100, 511, 512, 513, 1000, 2049]
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
-@pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 64)])
+@pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 64), (128, 8), (64, 24)])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (8, 1)])
 @pytest.mark.parametrize("part", [0, 512, 2048])
 def test_fused_append_decode_matches_append_then_decode(dt, D, B, Hq, Hkv, part):

@@ -26,7 +26,7 @@ EDGE_LENS = [1, 15, 16, 17, 31, 37, 63, 64, 65, 200, 513, 1100]
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("B", [16, 32])
+@pytest.mark.parametrize("B", [8, 16, 24, 32])  # 8, 24: a tile spans two blocks
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (8, 1), (16, 2)])
 @pytest.mark.parametrize("part", [0, 64, 512])
 def test_decode_16bit_matches_oracle(dt, D, B, Hq, Hkv, part):
@@ -86,19 +86,22 @@ def test_placement_invariance_and_contiguous_equality():
         assert torch.equal(o, outs[0])  # same arithmetic order: identical bits
 
 
-def test_zero_length_and_tail_poison():
-    c = make_random_case("zero", 4, 2, 128, 16, [0, 5, 16, 0, 33], torch.float16, seed=3,
-                         device=DEV, pool_blocks=10)
+@pytest.mark.parametrize("B", [16, 8])
+def test_zero_length_and_tail_poison(B):
+    c = make_random_case("zero", 4, 2, 128, B, [0, 5, 16, 0, 33], torch.float16, seed=3,
+                         device=DEV, pool_blocks=160 // B)
     got = gpu_decode(c, partition_size=16)
     assert torch.isnan(c.k_pool).any()  # poisoned slots exist
     assert (got[0] == 0).all() and (got[3] == 0).all()
     assert_close_to_oracle(got, oracle_decode(c), torch.float16, "zero/poison")
 
 
-def test_bad_block_id_reports_and_masks():
-    c = make_random_case("bad", 4, 4, 128, 16, [40, 20], torch.bfloat16, seed=9, device=DEV)
+@pytest.mark.parametrize("B,entry", [(16, 1), (8, 1), (8, 2)])
+def test_bad_block_id_reports_and_masks(B, entry):
+    # with B = 8, entry 1 is the second unit of tile 0 and entry 2 the first of tile 1
+    c = make_random_case("bad", 4, 4, 128, B, [40, 20], torch.bfloat16, seed=9, device=DEV)
     bt = c.block_tables.clone()
-    bt[0, 1] = c.num_blocks + 5
+    bt[0, entry] = c.num_blocks + 5
     c.block_tables = bt
     err = new_err(DEV)
     got = gpu_decode(c, err=err)
@@ -123,9 +126,9 @@ def test_host_checked_errors():
     with pytest.raises(pkv.PkvError) as e:
         gpu_decode(c, partition_size=24)
     assert e.value.status == pkv.PKV_EINVAL
-    c8 = make_random_case("b8", 4, 4, 128, 8, [20], torch.bfloat16, seed=2, device=DEV)
-    with pytest.raises(pkv.PkvError) as e:
-        gpu_decode(c8)
+    c12 = make_random_case("b12", 4, 4, 128, 12, [20], torch.bfloat16, seed=2, device=DEV)
+    with pytest.raises(pkv.PkvError) as e:  # 16-bit block sizes are multiples of 8
+        gpu_decode(c12)
     assert e.value.status == pkv.PKV_EUNSUPPORTED
 
 
