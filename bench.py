@@ -252,6 +252,49 @@ def step_bytes(case, nseq=None):
     return b, app
 
 
+def measure_swap(case, dev, stream, pkv, nseq=32, reps=5):
+    """Swap the blocks of the batch's first `nseq` sequences out to a swap
+    space in pinned host memory and back in (kv_block_swap, both directions),
+    as preemption does. Times each direction with CUDA events; the bound is
+    the host link, so the measured pinned copy rates are reported beside."""
+    import torch
+    B = case.block_size
+    lens = case.context_lens[:nseq].cpu().tolist()
+    bt = case.block_tables[:nseq].cpu()
+    blocks = sorted({int(b) for s, L in enumerate(lens) for b in bt[s, :-(-L // B)].tolist()})
+    n = len(blocks)
+    if n == 0:
+        return None
+    shape = (n,) + tuple(case.k_pool.shape[1:])
+    hk = torch.empty(shape, dtype=case.k_pool.dtype, pin_memory=True)
+    hv = torch.empty(shape, dtype=case.k_pool.dtype, pin_memory=True)
+    out_pairs = torch.tensor([[b, i] for i, b in enumerate(blocks)], dtype=torch.int32,
+                             device=dev)
+    in_pairs = out_pairs.flip(1).contiguous()
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    nbytes = 2 * n * case.k_pool[0].numel() * case.k_pool.element_size()
+
+    def timed(dst_k, dst_v, src_k, src_v, pairs):
+        ts = []
+        for _ in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            pkv.kv_block_swap(dst_k, dst_v, src_k, src_v, pairs, err=err)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts[1:])
+    out_ms = timed(hk, hv, case.k_pool, case.v_pool, out_pairs)
+    in_ms = timed(case.k_pool, case.v_pool, hk, hv, in_pairs)  # same data back in place
+    if int(err.item()) != 0:
+        raise RuntimeError("kv_block_swap reported a bad pair")
+    return {"sequences": nseq, "blocks": n, "bytes": nbytes,
+            "out_ms": out_ms, "out_gbs": nbytes / (out_ms * 1e-3) / 1e9,
+            "in_ms": in_ms, "in_gbs": nbytes / (in_ms * 1e-3) / 1e9,
+            "note": "device pool <-> swap space in pinned host memory, SM copies over the "
+                    "host link (no copy engine)"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -600,6 +643,8 @@ def run_ours(args, rank, world, local_rank):
     if int(err.item()) != 0:
         raise RuntimeError(f"device error word set: {pkv.device_error_message(int(err.item()))}")
 
+    swap = measure_swap(case, dev, stream, pkv) if args.workload != "shared_prefix" else None
+
     contiguous = None
     if args.contiguous and args.workload != "shared_prefix":
         ccase = make_case(args.workload, device=dev, with_append=False, placement="identity",
@@ -668,6 +713,9 @@ def run_ours(args, rank, world, local_rank):
     }
     if contiguous:
         line["paged_vs_contiguous"] = contiguous
+    if swap:
+        swap["pinned_h2d_gbs"], swap["pinned_d2h_gbs"] = h2d_gbs, d2h_gbs
+        line["swap"] = swap
     line["config"]["call"] = ("kv_cache_append + paged_attn_decode" if not fused else
                               "paged_attn_decode_append (append fused into the decode)")
     line.update(extras)

@@ -8,6 +8,8 @@
  *                      cached tokens, read through its block table
  *   kv_cache_append    scatter new tokens' K/V into their pool slots
  *   kv_block_copy      whole-block copies (copy-on-write of shared blocks)
+ *   kv_block_swap      whole-block copies between the device pools and a swap
+ *                      space in page-locked host memory
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -65,7 +67,7 @@ typedef enum { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
 enum {
   PKV_DEV_BAD_BLOCK = 1,     /* block-table entry outside [0, num_blocks) */
   PKV_DEV_BAD_SLOT = 2,      /* append slot >= num_blocks * block_size */
-  PKV_DEV_BAD_PAIR = 3,      /* copy pair with src or dst outside [0, num_blocks) */
+  PKV_DEV_BAD_PAIR = 3,      /* copy or swap pair with a block id outside its pool */
   PKV_DEV_CONTEXT_LEN = 4,   /* context_lens[s] > max_context_len or > table capacity */
   PKV_DEV_WAIT_TIMEOUT = 5,  /* an on-chip copy wait gave up (never expected) */
 };
@@ -244,6 +246,36 @@ int kv_cache_append(void *k_pool, void *v_pool, const void *k_new, const void *v
 int kv_block_copy(void *k_pool, void *v_pool, const int32_t *src_dst, int num_pairs,
                   int num_kv_heads, int head_dim, int block_size, int num_blocks, int dtype,
                   int32_t *err, void *stream);
+
+/*
+ * kv_block_swap - copy whole blocks between two pools of the same block shape:
+ * the device pools and a swap space in page-locked host memory, in either
+ * direction.
+ *
+ * For each pair i < num_pairs, (src, dst) = (src_dst[2i], src_dst[2i+1]), all
+ * num_kv_heads*block_size*head_dim elements of block src of (src_k, src_v)
+ * are copied to block dst of (dst_k, dst_v). This is the data half of
+ * swapping (page "PagedAttention Analysis", ryotta.opik.net, section 6): when
+ * memory runs short, the blocks of a preempted sequence are copied to CPU
+ * memory, which has its own block allocator, all of a sequence's blocks
+ * together; they are copied back when it resumes. The copy is bit-exact.
+ *
+ * dst_k, dst_v  [dst_blocks][num_kv_heads][block_size][head_dim]
+ * src_k, src_v  [src_blocks][num_kv_heads][block_size][head_dim]
+ *               Each of the four may be device memory or page-locked host
+ *               memory that the device addresses directly (unified
+ *               addressing); 16-byte aligned. The kernels move the data with
+ *               16-byte loads and stores over the bus, with no separate copy.
+ * src_dst       int32 [num_pairs][2], device or page-locked host memory.
+ *               Precondition: the dst blocks are distinct and the source and
+ *               destination regions do not overlap. A pair with src outside
+ *               [0, src_blocks) or dst outside [0, dst_blocks) is skipped and
+ *               reported in *err (PKV_DEV_BAD_PAIR).
+ */
+int kv_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                  const int32_t *src_dst, int num_pairs, int num_kv_heads, int head_dim,
+                  int block_size, int src_blocks, int dst_blocks, int dtype, int32_t *err,
+                  void *stream);
 
 /* Static, human-readable text for a pkv_status value. */
 const char *pkv_status_string(int status);

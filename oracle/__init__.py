@@ -55,6 +55,7 @@ def _load():
                                                         I, I, I, I, I, I, I, D, I, I]
         lib.oracle_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, I]
         lib.oracle_block_copy.argtypes = [P, P, P, I, I, I, I, I, I]
+        lib.oracle_block_swap.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I]
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_half_to_double.restype = D
         lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
@@ -62,7 +63,7 @@ def _load():
         lib.oracle_num_threads.restype = I
         for f in ("oracle_paged_decode", "oracle_paged_decode_blockwise",
                   "oracle_paged_decode_partitioned", "oracle_cache_append",
-                  "oracle_block_copy"):
+                  "oracle_block_copy", "oracle_block_swap"):
             getattr(lib, f).restype = I
         _lib = lib
     return _lib
@@ -176,6 +177,19 @@ def cache_append(k_pool, v_pool, k_new, v_new, slot_mapping) -> None:
     rc = lib.oracle_cache_append(_ptr(k_pool), _ptr(v_pool), _ptr(k_new), _ptr(v_new),
                                  _ptr(slot_mapping), T, Hkv, D, B, P, es)
     _check(rc, "cache_append")
+
+
+def block_swap(dst_k, dst_v, src_k, src_v, pairs) -> None:
+    """CPU whole-block copies from block src of the source pools into block
+    dst of the destination pools (K and V)."""
+    lib = _load()
+    Ps, Hkv, B, D = (int(x) for x in src_k.shape)
+    Pd = int(dst_k.shape[0])
+    _, es = _dtype_code(src_k)
+    n = int(pairs.shape[0]) if pairs.ndim == 2 else 0
+    rc = lib.oracle_block_swap(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), _ptr(pairs), n,
+                               Hkv, D, B, Ps, Pd, es)
+    _check(rc, "block_swap")
 
 
 def block_copy(k_pool, v_pool, pairs) -> None:

@@ -35,6 +35,10 @@
  *   oracle_block_copy          - page "추론 엔진에서의 메모리 가상화"
  *                                (molayo1419.me), copy-on-write section: the
  *                                old block's contents are copied to the new.
+ *   oracle_block_swap          - page "PagedAttention Analysis"
+ *                                (ryotta.opik.net), section 6: a preempted
+ *                                sequence's blocks are copied to blocks of a
+ *                                separate (CPU) pool and back.
  */
 #include <math.h>
 #include <stdint.h>
@@ -415,6 +419,32 @@ int oracle_block_copy(void *k_pool, void *v_pool, const int32_t *pairs, int num_
     memcpy((char *)k_pool + (size_t)dst * block_bytes, (const char *)k_pool + (size_t)src * block_bytes,
            block_bytes);
     memcpy((char *)v_pool + (size_t)dst * block_bytes, (const char *)v_pool + (size_t)src * block_bytes,
+           block_bytes);
+  }
+  return status;
+}
+
+/*
+ * Block swap: for each pair (src, dst), the whole block src of the source
+ * pools is copied into block dst of the destination pools (both K and V).
+ * Out-of-range ids (src against src_blocks, dst against dst_blocks) are an
+ * error, and that pair is skipped.
+ */
+int oracle_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                      const int32_t *pairs, int num_pairs, int Hkv, int D, int B,
+                      int src_blocks, int dst_blocks, int elem_bytes) {
+  if (num_pairs < 0 || Hkv <= 0 || D <= 0 || B <= 0 || elem_bytes <= 0) return ORACLE_EBADARG;
+  int status = ORACLE_OK;
+  size_t block_bytes = (size_t)Hkv * B * D * elem_bytes;
+  for (int i = 0; i < num_pairs; ++i) {
+    int src = pairs[2 * i], dst = pairs[2 * i + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+      status = ORACLE_EBADBLOCK;
+      continue;
+    }
+    memcpy((char *)dst_k + (size_t)dst * block_bytes, (const char *)src_k + (size_t)src * block_bytes,
+           block_bytes);
+    memcpy((char *)dst_v + (size_t)dst * block_bytes, (const char *)src_v + (size_t)src * block_bytes,
            block_bytes);
   }
   return status;

@@ -24,13 +24,13 @@ LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
 PKV_OK, PKV_EINVAL, PKV_EUNSUPPORTED, PKV_ECUDA = 0, -1, -2, -3
 DEV_ERRORS = {1: "block id out of range", 2: "append slot out of range",
-              3: "copy pair out of range", 4: "context length above max_context_len",
+              3: "copy or swap pair out of range", 4: "context length above max_context_len",
               5: "copy wait timed out"}
 DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DEFAULT_PARTITION = 2048  # tokens per split-context partition (measured best on B200)
 
 EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
-           "kv_block_copy", "pkv_decode_workspace_bytes", "pkv_status_string")
+           "kv_block_copy", "kv_block_swap", "pkv_decode_workspace_bytes", "pkv_status_string")
 
 
 class PkvError(RuntimeError):
@@ -62,6 +62,8 @@ def load_library():
     lib.kv_cache_append.restype = I
     lib.kv_block_copy.argtypes = [P, P, P, I, I, I, I, I, I, P, P]
     lib.kv_block_copy.restype = I
+    lib.kv_block_swap.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P]
+    lib.kv_block_swap.restype = I
     lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_bytes.restype = Z
     lib.pkv_status_string.argtypes = [I]
@@ -226,6 +228,50 @@ def kv_block_copy(k_pool: torch.Tensor, v_pool: torch.Tensor, src_dst: torch.Ten
                            DTYPE_CODES[k_pool.dtype], _dev_ptr(err, "err", dev),
                            _stream_ptr(stream, dev))
     _check("kv_block_copy", rc)
+
+
+def _dev_or_pinned_ptr(t: torch.Tensor, name: str, device):
+    """A CUDA tensor on `device`, or a page-locked host tensor the device can
+    address directly."""
+    if isinstance(t, torch.Tensor) and t.device.type == "cpu":
+        if not t.is_pinned():
+            raise ValueError(f"{name} on the host must be pinned (page-locked) memory")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        return ctypes.c_void_p(t.data_ptr())
+    return _dev_ptr(t, name, device)
+
+
+def kv_block_swap(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                  src_v: torch.Tensor, src_dst: torch.Tensor, err: Optional[torch.Tensor] = None,
+                  stream=None, device=None) -> None:
+    """Copy whole blocks ``src_dst[i] = (src, dst)`` (int32 [N][2]) from the
+    source pools to the destination pools. Each pool, and ``src_dst``, may be
+    on the GPU or in pinned host memory: swap-out is device -> host, swap-in
+    host -> device."""
+    lib = load_library()
+    if device is None:
+        cuda = [t for t in (dst_k, dst_v, src_k, src_v, src_dst) if t.device.type == "cuda"]
+        device = cuda[0].device if cuda else torch.device("cuda", torch.cuda.current_device())
+    dt = src_k.dtype
+    if dt not in DTYPE_CODES or any(t.dtype != dt for t in (src_v, dst_k, dst_v)):
+        raise TypeError("pools must share one of float32/float16/bfloat16")
+    if src_dst.dtype != torch.int32:
+        raise TypeError("src_dst must be int32")
+    Ps, Hkv, B, D = (int(x) for x in src_k.shape)
+    Pd = int(dst_k.shape[0])
+    if tuple(src_v.shape) != (Ps, Hkv, B, D) or tuple(dst_k.shape[1:]) != (Hkv, B, D) \
+            or tuple(dst_v.shape) != (Pd, Hkv, B, D):
+        raise ValueError("pools must share the block shape [Hkv][B][D]")
+    N = int(src_dst.shape[0]) if src_dst.numel() else 0
+    if N and tuple(src_dst.shape) != (N, 2):
+        raise ValueError("src_dst must be [N][2]")
+    ptr = lambda t, n: _dev_or_pinned_ptr(t, n, device)
+    rc = lib.kv_block_swap(ptr(dst_k, "dst_k"), ptr(dst_v, "dst_v"), ptr(src_k, "src_k"),
+                           ptr(src_v, "src_v"), ptr(src_dst, "src_dst") if N else None, N, Hkv,
+                           D, B, Ps, Pd, DTYPE_CODES[dt], _dev_ptr(err, "err", device),
+                           _stream_ptr(stream, device))
+    _check("kv_block_swap", rc)
 
 
 def device_error_message(code: int) -> str:

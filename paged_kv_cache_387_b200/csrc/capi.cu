@@ -304,4 +304,25 @@ int kv_block_copy(void *k_pool, void *v_pool, const int32_t *src_dst, int num_pa
                                             num_blocks, err, static_cast<cudaStream_t>(stream)));
 }
 
+int kv_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                  const int32_t *src_dst, int num_pairs, int num_kv_heads, int head_dim,
+                  int block_size, int src_blocks, int dst_blocks, int dtype, int32_t *err,
+                  void *stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      src_blocks <= 0 || dst_blocks <= 0)
+    return PKV_EINVAL;
+  if (dtype < PKV_F32 || dtype > PKV_BF16) return PKV_EINVAL;
+  if (num_pairs == 0) return PKV_OK;
+  if (!dst_k || !dst_v || !src_k || !src_v || !src_dst) return PKV_EINVAL;
+  const int es = dtype == PKV_F32 ? 4 : 2;
+  const long long block_bytes = (long long)num_kv_heads * block_size * head_dim * es;
+  if (((long long)head_dim * es) % 16 != 0) return PKV_EUNSUPPORTED;
+  if (!aligned(dst_k, 16) || !aligned(dst_v, 16) || !aligned(src_k, 16) || !aligned(src_v, 16) ||
+      !aligned(src_dst, 4))
+    return PKV_EINVAL;
+  return cuda_status(pkv::launch_block_swap(dst_k, dst_v, src_k, src_v, src_dst, num_pairs,
+                                            block_bytes, src_blocks, dst_blocks, err,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -69,6 +69,9 @@ cudaError_t launch_merge(const DecodeArgs &a, int dtype, cudaStream_t stream);
 cudaError_t launch_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,
                           const int64_t *slots, int num_tokens, int num_kv_heads, int row_bytes,
                           int block_size, int num_blocks, int32_t *err, cudaStream_t stream);
+cudaError_t launch_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                              const int32_t *pairs, int num_pairs, long long block_bytes,
+                              int src_blocks, int dst_blocks, int32_t *err, cudaStream_t stream);
 cudaError_t launch_block_copy(void *k_pool, void *v_pool, const int32_t *pairs, int num_pairs,
                               long long block_bytes, int num_blocks, int32_t *err,
                               cudaStream_t stream);

@@ -16,7 +16,7 @@ Modules:
 * ``accounting`` - byte counts used for the bandwidth figures.
 """
 
-from .block_manager import BlockAllocator, CowCopy  # noqa: F401
+from .block_manager import BlockAllocator, BlockMove, CowCopy, SeqState, SwapSpace  # noqa: F401
 from .workloads import (  # noqa: F401
     DecodeCase,
     POOL_LAYOUT,

@@ -21,6 +21,12 @@ What it follows:
   writes into the partially filled shared block gets a new block (#45). The
   contents are copied, that branch's table entry is repointed, and the old
   block's refcount drops by one.
+* page "PagedAttention Analysis" (ryotta.opik.net), section 6, for swapping.
+  Beside the GPU block allocator sits a CPU one. A preempted sequence's blocks
+  are copied to CPU blocks, all of the sequence's blocks together or none
+  (all-or-nothing). The swap space never holds more blocks than the GPU pool
+  has, which bounds it. The moves this returns are executed by the
+  ``kv_block_swap`` kernel (or by the oracle's block swap).
 
 Allocation only updates integer indices on the host. It never touches device
 memory, which matches the pages' point that block management needs no
@@ -29,6 +35,7 @@ memory, which matches the pages' point that block management needs no
 
 from __future__ import annotations
 
+from collections import Counter
 from dataclasses import dataclass, field
 from typing import List, Optional, Sequence, Tuple
 
@@ -43,12 +50,24 @@ class CowCopy:
     dst: int
 
 
+@dataclass(frozen=True)
+class BlockMove:
+    """One whole-block copy from block ``src`` of one pool to block ``dst`` of another."""
+
+    src: int
+    dst: int
+
+
 @dataclass
 class SeqState:
-    """A sequence's block table (logical -> physical) and its token count."""
+    """A sequence's block table (logical -> physical) and its token count.
+
+    ``on_host`` tells which pool the table's ids refer to: the GPU pool, or the
+    swap space after the sequence was swapped out."""
 
     table: List[int] = field(default_factory=list)
     num_tokens: int = 0
+    on_host: bool = False
 
 
 class BlockAllocator:
@@ -100,7 +119,21 @@ class BlockAllocator:
         if self._ref[block] == 0:
             self._free.append(block)
 
+    def reference(self, block: int) -> None:
+        """Add a reference to a block, taking it off the free list if it was free."""
+        if self._ref[block] == 0:
+            self._free.remove(block)
+        self._ref[block] += 1
+
     # -- sequence-level operations -------------------------------------------
+    def adopt(self, table: Sequence[int], num_tokens: int) -> SeqState:
+        """Take over an existing block table (one reference per entry)."""
+        if -(-int(num_tokens) // self.block_size) != len(table):
+            raise ValueError("table length does not match the token count")
+        for b in table:
+            self.reference(int(b))
+        return SeqState(table=[int(b) for b in table], num_tokens=int(num_tokens))
+
     def new_sequence(self, num_tokens: int) -> SeqState:
         """Attach ceil(num_tokens / B) fresh blocks for a prompt."""
         seq = SeqState()
@@ -148,3 +181,60 @@ class BlockAllocator:
     def waste_slots(seq: SeqState, block_size: int) -> int:
         """Reserved but unfilled slots of a sequence (its last block only)."""
         return len(seq.table) * block_size - seq.num_tokens
+
+
+class SwapSpace:
+    """A CPU block allocator beside a GPU one, for swapping preempted sequences.
+
+    ``swap_out`` moves every block of a group of sequences (for example the
+    samples of one request, which may share blocks) into the swap space, and
+    ``swap_in`` moves them back into the GPU pool. Both are all-or-nothing: if
+    the target allocator cannot hold every distinct block of the group, nothing
+    changes and MemoryError is raised. A block shared within the group moves
+    once, and its refcount on the other side equals the number of table
+    entries that reference it. The swap space is bounded by the GPU pool's
+    block count.
+    """
+
+    def __init__(self, gpu: BlockAllocator, num_cpu_blocks: Optional[int] = None):
+        n = gpu.num_blocks if num_cpu_blocks is None else int(num_cpu_blocks)
+        if n > gpu.num_blocks:
+            raise ValueError("the swap space holds at most as many blocks as the GPU pool")
+        self.gpu = gpu
+        self.cpu = BlockAllocator(n, gpu.block_size)
+
+    def _move(self, seqs: Sequence[SeqState], src: BlockAllocator, dst: BlockAllocator,
+              to_host: bool) -> List[BlockMove]:
+        if any(sq.on_host == to_host for sq in seqs):
+            raise ValueError("every sequence of the group must be on the source side")
+        distinct: List[int] = []  # the group's source blocks, in first-use order
+        seen = set()
+        for sq in seqs:
+            for b in sq.table:
+                if b not in seen:
+                    seen.add(b)
+                    distinct.append(b)
+        if len(distinct) > dst.num_free:
+            raise MemoryError("not enough free blocks for the whole group")
+        mapping = {b: dst.allocate() for b in distinct}  # one reference each
+        for sq in seqs:
+            old = sq.table
+            sq.table = [mapping[b] for b in old]
+            sq.on_host = to_host
+            for b in old:  # the group's references leave the source side
+                src.free(b)
+        # one reference per table entry on the destination side
+        counts = Counter(nb for sq in seqs for nb in sq.table)
+        for nb, c in counts.items():
+            for _ in range(c - 1):
+                dst.reference(nb)
+        return [BlockMove(src=b, dst=mapping[b]) for b in distinct]
+
+    def swap_out(self, seqs: Sequence[SeqState]) -> List[BlockMove]:
+        """GPU -> swap space. Returns the moves (GPU block -> CPU block). The
+        moves must run before the freed GPU blocks are handed out again."""
+        return self._move(seqs, self.gpu, self.cpu, True)
+
+    def swap_in(self, seqs: Sequence[SeqState]) -> List[BlockMove]:
+        """Swap space -> GPU. Returns the moves (CPU block -> GPU block)."""
+        return self._move(seqs, self.cpu, self.gpu, False)

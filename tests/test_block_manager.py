@@ -101,3 +101,86 @@ def test_shared_prefix_copies_follow_refcount_rule():
     bt = st["block_tables"]
     assert (bt[0, :2] == bt[1, :2]).all() and (bt[0, :2] == bt[2, :2]).all()
     assert bt[0, 2] != bt[1, 2] != bt[2, 2]
+
+
+# ---------------------------------------------------------------------------
+# swapping (page "PagedAttention Analysis", section 6): a CPU block allocator
+# beside the GPU one, all-or-nothing moves, swap space bounded by the GPU pool
+# ---------------------------------------------------------------------------
+
+from pkv_inputs import SwapSpace  # noqa: E402
+
+
+def _sharing_pattern(seqs):
+    """Which table positions hold the same block (the ids themselves may differ)."""
+    ids = [b for sq in seqs for b in sq.table]
+    first = {}
+    return [first.setdefault(b, i) for i, b in enumerate(ids)]
+
+
+def test_swap_space_is_bounded_by_the_gpu_pool():
+    gpu = BlockAllocator(10, 16)
+    with pytest.raises(ValueError):
+        SwapSpace(gpu, 11)
+    assert SwapSpace(gpu).cpu.num_blocks == 10
+
+
+def test_swap_out_is_all_or_nothing():
+    gpu = BlockAllocator(20, 16)
+    sw = SwapSpace(gpu, 4)
+    a = gpu.new_sequence(70)  # 5 blocks > 4 free in the swap space
+    before = (list(a.table), gpu.num_free, sw.cpu.num_free)
+    with pytest.raises(MemoryError):
+        sw.swap_out([a])
+    assert (a.table, gpu.num_free, sw.cpu.num_free) == before and not a.on_host
+
+
+def test_swap_round_trip_keeps_sharing_and_refcounts():
+    B = 16
+    gpu = BlockAllocator(40, B, free_order=np.random.default_rng(5).permutation(40))
+    sw = SwapSpace(gpu)
+    prompt = gpu.new_sequence(40)  # 2 full blocks + 1 partial
+    samples = [prompt] + [gpu.fork(prompt) for _ in range(2)]
+    for sq in samples:  # each sample writes one token: copy-on-write of the partial block
+        gpu.append_slot(sq)
+    pattern = _sharing_pattern(samples)
+    distinct = len(set(b for sq in samples for b in sq.table))
+    gpu_free0 = gpu.num_free
+    moves = sw.swap_out(samples)
+    assert len(moves) == distinct and len({m.src for m in moves}) == distinct
+    assert all(sq.on_host for sq in samples)
+    assert gpu.num_free == gpu_free0 + distinct  # nothing else referenced them
+    assert _sharing_pattern(samples) == pattern
+    shared = samples[0].table[0]
+    assert sw.cpu.refcount(shared) == 3  # one reference per table entry
+    # the moves map each GPU block to the CPU block that replaced it
+    m = {mv.src: mv.dst for mv in moves}
+    assert len(set(m.values())) == distinct
+    back = sw.swap_in(samples)
+    assert len(back) == distinct and not any(sq.on_host for sq in samples)
+    assert sw.cpu.num_free == sw.cpu.num_blocks and gpu.num_free == gpu_free0
+    assert _sharing_pattern(samples) == pattern
+    assert gpu.refcount(samples[1].table[0]) == 3
+
+
+def test_swap_out_copies_blocks_still_referenced_outside_the_group():
+    gpu = BlockAllocator(12, 16)
+    sw = SwapSpace(gpu)
+    a = gpu.new_sequence(32)
+    b = gpu.fork(a)  # b stays on the GPU
+    moves = sw.swap_out([a])
+    assert len(moves) == 2
+    assert [gpu.refcount(x) for x in b.table] == [1, 1]  # still owned by b
+    assert gpu.num_free == 10
+    with pytest.raises(ValueError):
+        sw.swap_out([a])  # already on the host
+
+
+def test_adopt_takes_over_existing_tables():
+    gpu = BlockAllocator(8, 16)
+    sq = gpu.adopt([5, 2], 20)
+    assert gpu.num_free == 6 and gpu.refcount(5) == 1
+    other = gpu.adopt([5], 3)  # a shared first block
+    assert gpu.refcount(5) == 2 and other.table == [5]
+    with pytest.raises(ValueError):
+        gpu.adopt([1], 40)  # 40 tokens need 3 blocks

@@ -254,3 +254,26 @@ def test_block_copy_matches_numpy_slices():
     oracle.block_copy(k_pool, v_pool, torch.from_numpy(pairs))
     assert np.array_equal(k_pool.view(torch.int16).numpy(), ek)
     assert np.array_equal(v_pool.view(torch.int16).numpy(), ev)
+
+
+def test_block_swap_is_numpy_block_assignment():
+    """oracle.block_swap copies whole blocks between two pools: the same as
+    torch's indexed assignment dst[d] = src[s] per pair, bit for bit."""
+    import torch
+    rng = np.random.default_rng(11)
+    for dt in (torch.float16, torch.bfloat16, torch.float32):
+        src_k = torch.from_numpy(rng.standard_normal((9, 2, 16, 64)).astype(np.float32)).to(dt)
+        src_v = torch.from_numpy(rng.standard_normal((9, 2, 16, 64)).astype(np.float32)).to(dt)
+        dst_k = torch.full((6, 2, 16, 64), float("nan"), dtype=dt)
+        dst_v = torch.full_like(dst_k, float("nan"))
+        pairs = np.array([[7, 0], [2, 5], [7, 3], [0, 1]], dtype=np.int32)
+        ek, ev = dst_k.clone(), dst_v.clone()
+        for s_, d_ in pairs:
+            ek[d_] = src_k[s_]
+            ev[d_] = src_v[s_]
+        oracle.block_swap(dst_k, dst_v, src_k, src_v, pairs)
+        bits = torch.int32 if dt == torch.float32 else torch.int16
+        assert torch.equal(dst_k.view(bits), ek.view(bits))
+        assert torch.equal(dst_v.view(bits), ev.view(bits))
+        with pytest.raises(RuntimeError):
+            oracle.block_swap(dst_k, dst_v, src_k, src_v, np.array([[9, 0]], dtype=np.int32))
