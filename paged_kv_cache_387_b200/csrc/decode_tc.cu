@@ -133,14 +133,20 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
 //  2. Sequences of one partition, ordered by size, largest first (a counting
 //     sort over PLAN_BUCKETS size classes). They need no merge, and handing out
 //     the largest first and the smallest last keeps the CTAs' finishing times
-//     close. A sequence of length 0 is one (empty) entry, so that its output is
-//     still written.
-// Each entry carries the sequence's clamped length. The merge counters are
-// reset here too.
+//     close. The sort is stable: within a size class the sequences keep their
+//     order, so sequences that share blocks and sit next to each other in the
+//     batch (the samples of one prompt) are attended together, and their shared
+//     blocks are fetched once and then served from L2. A sequence of length 0 is
+//     one (empty) entry, so that its output is still written.
+// Each entry carries the sequence's clamped length. Sequences are taken in
+// rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t), so
+// that thread order is sequence order. The merge counters are reset here too.
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
   constexpr int NW = PLAN_THREADS / 32;
   __shared__ int wsum[NW];
-  __shared__ int hist[PLAN_BUCKETS];
+  __shared__ int hist[PLAN_BUCKETS];        // count, then running start of each size class
+  __shared__ int wcnt[NW][PLAN_BUCKETS];    // per-warp counts of a round, then their offsets
+  __shared__ int total_m_s;
   pdl_launch_dependents();  // the decode grid may launch; it waits for this grid to finish
   // This grid may itself start while the previous decode call is finishing:
   // nothing in global memory is touched before that call has completed.
@@ -154,46 +160,54 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   }
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
   __syncthreads();
-  const int chunk = (S + PLAN_THREADS - 1) / PLAN_THREADS;
-  const int s0 = min(S, tid * chunk), s1 = min(S, s0 + chunk);
   const int max_tiles = max(1, P / 16);
-  // size class of a one-partition sequence of `len` tokens: bigger -> smaller bucket
+  // size class of a one-partition sequence of `len` tokens: bigger -> smaller class
   auto bucket = [&](int len) {
     const int tiles = (len + 15) / 16;
     return (PLAN_BUCKETS - 1) - min(PLAN_BUCKETS - 1, tiles * (PLAN_BUCKETS - 1) / max_tiles);
   };
-
-  int nm = 0;  // region-1 entries of this thread's sequences
-  for (int s = s0; s < s1; ++s) {
-    const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
-                                a.block_size, a.err);
-    if (L > P)
-      nm += (L + P - 1) / P;
-    else
-      atomicAdd(&hist[bucket(L)], 1);
-  }
-  // block-wide exclusive scan of the region-1 counts
-  int f = nm;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(FULL_MASK, f, off);
-    if (lane >= off) f += y;
-  }
-  if (lane == 31) wsum[warp] = f;
-  __syncthreads();
-  if (warp == 0) {
-    int v = lane < NW ? wsum[lane] : 0;
+  // Exclusive block-wide prefix sum of v; `total` receives the sum.
+  auto block_scan = [&](int v, int &total) {
+    int f = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(FULL_MASK, v, off);
-      if (lane >= off) v += y;
+      const int y = __shfl_up_sync(FULL_MASK, f, off);
+      if (lane >= off) f += y;
     }
-    if (lane < NW) wsum[lane] = v;  // inclusive prefix over warps
+    if (lane == 31) wsum[warp] = f;
+    __syncthreads();
+    if (warp == 0) {
+      int w = lane < NW ? wsum[lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, w, off);
+        if (lane >= off) w += y;
+      }
+      if (lane < NW) wsum[lane] = w;  // inclusive prefix over warps
+    }
+    __syncthreads();
+    const int excl = (warp ? wsum[warp - 1] : 0) + f - v;
+    total = wsum[NW - 1];
+    __syncthreads();  // wsum is reused by the next scan
+    return excl;
+  };
+
+  // pass 1: region-1 entry count and the size-class histogram of region 2
+  int nm = 0;
+  for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
+    const int s = r0 + tid;
+    if (s < S) {
+      const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
+                                  a.block_size, a.err);
+      if (L > P)
+        nm += (L + P - 1) / P;
+      else
+        atomicAdd(&hist[bucket(L)], 1);
+    }
   }
-  __syncthreads();
-  const int base_m = (warp ? wsum[warp - 1] : 0) + f - nm;
-  const int total_m = wsum[NW - 1];
-  // bucket offsets (exclusive scan of hist, after region 1)
+  int total_m;
+  block_scan(nm, total_m);
+  // running start of each size class (exclusive scan of hist, after region 1)
   if (warp == 0) {
     const int h0 = hist[2 * lane], h1 = hist[2 * lane + 1];
     int v = h0 + h1;
@@ -205,24 +219,54 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     const int excl = v - h0 - h1;
     hist[2 * lane] = total_m + excl;
     hist[2 * lane + 1] = total_m + excl + h0;
-    if (lane == 31 && tid == 31) {
+    if (lane == 31) {
       a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
       a.sched[1] = total_m + v;
     }
   }
+  if (tid == 0) total_m_s = 0;
   __syncthreads();
 
-  int om = base_m;
-  for (int s = s0; s < s1; ++s) {
-    const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
-                                a.block_size, nullptr);
-    if (L > P) {
-      const int np = (L + P - 1) / P;
-      a.work[om++] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
-      for (int q = 0; q < np - 1; ++q) a.work[om++] = make_uint2(pack_pair(s, q), (uint32_t)L);
-    } else {
-      a.work[atomicAdd(&hist[bucket(L)], 1)] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+  // pass 2: write the entries, one round of PLAN_THREADS sequences at a time
+  for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
+    const int s = r0 + tid;
+    int L = 0, np = 0, bkt = -1;
+    if (s < S) {
+      L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, a.block_size,
+                        nullptr);
+      if (L > P)
+        np = (L + P - 1) / P;
+      else
+        bkt = bucket(L);
     }
+    // region 1: this round's entries after the previous rounds'
+    int round_m;
+    const int om = total_m_s + block_scan(np, round_m);
+    if (np > 0) {
+      a.work[om] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
+      for (int q = 0; q < np - 1; ++q) a.work[om + 1 + q] = make_uint2(pack_pair(s, q), (uint32_t)L);
+    }
+    // region 2: rank among this warp's lanes of the same class, then the
+    // earlier warps' counts, then the class's running start
+    for (int i = tid; i < NW * PLAN_BUCKETS; i += PLAN_THREADS) (&wcnt[0][0])[i] = 0;
+    __syncthreads();
+    const unsigned same = __match_any_sync(FULL_MASK, bkt);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    if (bkt >= 0 && lane == 31 - __clz(same)) wcnt[warp][bkt] = __popc(same);
+    __syncthreads();
+    if (tid < PLAN_BUCKETS) {
+      int start = hist[tid];
+      for (int w = 0; w < NW; ++w) {
+        const int c = wcnt[w][tid];
+        wcnt[w][tid] = start;
+        start += c;
+      }
+      hist[tid] = start;
+    }
+    if (tid == 0) total_m_s += round_m;
+    __syncthreads();
+    if (bkt >= 0) a.work[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+    __syncthreads();  // wcnt and total_m_s are rewritten by the next round
   }
 }
 
@@ -491,6 +535,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       int next = 0;
       if (prefetch && lane == 0) next = atomicAdd(&a.sched[0], 1);
 
+      // Items are entry-major: the KV heads of one entry are consecutive items.
+      // A block's heads are contiguous in the pool, so CTAs working on
+      // neighbouring items read neighbouring 4 KB slices (open DRAM rows).
       const uint2 wk = a.work[item / Hkv];
       const int h = item - (item / Hkv) * Hkv;
       const int s = min(static_cast<int>(wk.x >> 16), a.num_seqs - 1);
