@@ -261,7 +261,16 @@ def measure_swap(case, dev, stream, pkv, nseq=32, reps=5):
     B = case.block_size
     lens = case.context_lens[:nseq].cpu().tolist()
     bt = case.block_tables[:nseq].cpu()
-    blocks = sorted({int(b) for s, L in enumerate(lens) for b in bt[s, :-(-L // B)].tolist()})
+    blk_bytes = 2 * case.k_pool[0].numel() * case.k_pool.element_size()
+    blocks, seen = [], set()
+    for s, L in enumerate(lens):  # whole sequences, up to ~128 MB
+        if blocks and len(blocks) * blk_bytes >= (128 << 20):
+            nseq = s
+            break
+        for b in bt[s, :-(-L // B)].tolist():
+            if b not in seen:
+                seen.add(b)
+                blocks.append(int(b))
     n = len(blocks)
     if n == 0:
         return None
@@ -288,7 +297,7 @@ def measure_swap(case, dev, stream, pkv, nseq=32, reps=5):
     in_ms = timed(case.k_pool, case.v_pool, hk, hv, in_pairs)  # same data back in place
     if int(err.item()) != 0:
         raise RuntimeError("kv_block_swap reported a bad pair")
-    return {"sequences": nseq, "blocks": n, "bytes": nbytes,
+    return {"sequences": min(nseq, len(lens)), "blocks": n, "bytes": nbytes,
             "out_ms": out_ms, "out_gbs": nbytes / (out_ms * 1e-3) / 1e9,
             "in_ms": in_ms, "in_gbs": nbytes / (in_ms * 1e-3) / 1e9,
             "note": "device pool <-> swap space in pinned host memory, SM copies over the "
@@ -339,7 +348,10 @@ def config_block(case, workload, n_gpus):
         "desc", "shared prefix / parallel sampling: 16 prompts x 6 samples, 40 heads MHA, "
                 "head_dim 128, fp16, block 16, prompt 1000 tokens shared through refcounted "
                 "blocks, CoW copy of the partial block, then 64 divergent decode tokens "
-                "(the timed step is the 64th)" if workload == "shared_prefix" else workload)
+                "(the timed step is the 64th)" if workload == "shared_prefix" else
+        "beam search: 32 requests x 4 beams, 32 q heads / 8 kv heads, head_dim 128, bf16, "
+        "block 16, prompt 512, seeded random parents each step; the timed step is the 128th "
+        "(append + decode of the 128 beams)" if workload == "beam_search" else workload)
     return {
         "workload": workload, "desc": desc, "num_seqs_per_gpu": case.num_seqs,
         "num_heads": case.num_heads, "num_kv_heads": case.num_kv_heads,
@@ -364,6 +376,25 @@ def build_bench_case(args, dev, rank):
     import torch
     from pkv_inputs import make_case
     from pkv_inputs.workloads import WORKLOADS, DecodeCase, make_shared_prefix_case
+    if args.workload == "beam_search":
+        # 32 requests x 4 beams, Llama-8B-shaped heads: after 127 steps with seeded
+        # random parents, the timed step is the 128th (copies applied, then the
+        # fused append + decode of all 128 beams).
+        from pkv_inputs import make_beam_search_case
+        case = make_beam_search_case(device=dev, seed=rank_seed(393, rank))
+        m = case.meta
+        per_tok = 2 * case.num_kv_heads * case.head_dim * case.k_pool.element_size()
+        per_blk = per_tok * case.block_size
+        extras = {"beam_search": {
+            "requests": m["requests"], "width": m["width"],
+            "blocks_in_use": m["blocks_in_use"], "blocks_unshared": m["blocks_unshared"],
+            "memory_saving": 1.0 - m["blocks_in_use"] / m["blocks_unshared"],
+            "logical_kv_bytes": int(case.context_lens.sum()) * per_tok,
+            "unique_kv_bytes": m["blocks_in_use"] * per_blk,
+            "note": "value/roofline count logical bytes; blocks shared by the beams of a "
+                    "request are read from L2"}}
+        case.meta = {k: v for k, v in m.items() if k not in ("allocator", "searches")}
+        return case, extras
     if args.workload != "shared_prefix":
         case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
                          seed=rank_seed(WORKLOADS[args.workload]["seed"], rank))
@@ -719,6 +750,9 @@ def run_ours(args, rank, world, local_rank):
     line["config"]["call"] = ("kv_cache_append + paged_attn_decode" if not fused else
                               "paged_attn_decode_append (append fused into the decode)")
     line.update(extras)
+    if "beam_search" in extras:
+        bx = extras["beam_search"]
+        bx["unique_gbs"] = bx["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
     if "shared_prefix" in extras:
         sp_x = extras["shared_prefix"]
         sp_x["unique_gbs"] = sp_x["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9

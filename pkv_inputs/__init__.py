@@ -16,8 +16,10 @@ Modules:
 * ``accounting`` - byte counts used for the bandwidth figures.
 """
 
-from .block_manager import BlockAllocator, BlockMove, CowCopy, SeqState, SwapSpace  # noqa: F401
+from .block_manager import (  # noqa: F401
+    BeamSearch, BlockAllocator, BlockMove, CowCopy, SeqState, SwapSpace)
 from .workloads import (  # noqa: F401
+    make_beam_search_case,
     DecodeCase,
     POOL_LAYOUT,
     WORKLOADS,

@@ -238,3 +238,52 @@ class SwapSpace:
     def swap_in(self, seqs: Sequence[SeqState]) -> List[BlockMove]:
         """Swap space -> GPU. Returns the moves (CPU block -> GPU block)."""
         return self._move(seqs, self.cpu, self.gpu, False)
+
+
+class BeamSearch:
+    """The block bookkeeping of beam search for one request (page "PagedAttention
+    Analysis", ryotta.opik.net, section 4: the beams share the prompt and
+    intermediate blocks, and which blocks they share changes every step).
+
+    Each ``step`` takes, for every new beam, the index of the surviving beam it
+    continues. The new beams fork their parents (sharing every block by
+    reference), the old beams are released, and each beam then takes the slot
+    of its next token, copying its last block first when that block is shared.
+    """
+
+    def __init__(self, alloc: BlockAllocator, prompt_tokens: int, width: int):
+        if width <= 0:
+            raise ValueError("width must be positive")
+        self.alloc = alloc
+        root = alloc.new_sequence(prompt_tokens)
+        self.beams: List[SeqState] = [root] + [alloc.fork(root) for _ in range(width - 1)]
+
+    def step(self, parents: Sequence[int]) -> Tuple[List[int], List[CowCopy]]:
+        """Returns the slots of the beams' next tokens and the block copies to
+        run before those tokens are written."""
+        if len(parents) != len(self.beams):
+            raise ValueError("one parent per beam")
+        new = [self.alloc.fork(self.beams[int(p)]) for p in parents]
+        for b in self.beams:
+            self.alloc.release(b)
+        self.beams = new
+        slots: List[int] = []
+        copies: List[CowCopy] = []
+        for b in self.beams:
+            slot, cow = self.alloc.append_slot(b)
+            slots.append(slot)
+            if cow is not None:
+                copies.append(cow)
+        return slots, copies
+
+    def blocks_in_use(self) -> int:
+        return len({blk for b in self.beams for blk in b.table})
+
+    def blocks_unshared(self) -> int:
+        """Blocks the beams would hold without sharing (one table each)."""
+        return sum(len(b.table) for b in self.beams)
+
+    def release(self) -> None:
+        for b in self.beams:
+            self.alloc.release(b)
+        self.beams = []

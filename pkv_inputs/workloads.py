@@ -32,7 +32,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 import torch
 
-from .block_manager import BlockAllocator
+from .block_manager import BeamSearch, BlockAllocator
 
 POOL_LAYOUT = "[num_blocks][num_kv_heads][block_size][head_dim], head_dim contiguous"
 
@@ -399,3 +399,90 @@ def make_shared_prefix_case(device="cpu", seed: int = 391, num_prompts: int = 16
                             num_prompts=num_prompts, samples=samples,
                             prompt_len=prompt_len,
                             meta={"pool_blocks": P, "copies": len(cow)})
+
+
+def make_beam_search_case(device="cpu", seed: int = 393, num_requests: int = 32, width: int = 4,
+                          prompt_len: int = 512, steps: int = 127, num_heads: int = 32,
+                          num_kv_heads: int = 8, head_dim: int = 128, block_size: int = 16,
+                          dtype=torch.bfloat16, partition_size: int = DEFAULT_PARTITION):
+    """Beam search over ``num_requests`` requests of ``width`` beams (page
+    "PagedAttention Analysis", section 4: the beams share the prompt and
+    intermediate blocks, and the sharing changes every step).
+
+    Every step each request's new beams continue seeded random parents; the
+    copy-on-write block copies and the new tokens' K/V (N(0,1)) are applied to
+    the pools. After ``steps`` steps, the returned case is the next step: its
+    copies already applied, ``k_new``/``v_new``/``slot_mapping`` the tokens it
+    appends, and ``context_lens`` counting them. Sharing statistics are in
+    ``meta``: the blocks the beams hold, the blocks they would hold unshared.
+    """
+    B = block_size
+    rng = np.random.default_rng(seed)
+    gen = _generator(seed, device)
+    per_req = width * (-(-(prompt_len + steps + 1) // B) + 1)  # bound without sharing
+    P = num_requests * per_req
+    alloc = BlockAllocator(P, B, free_order=rng.permutation(P).tolist())
+    fill = float("nan")
+    k_pool = torch.full((P, num_kv_heads, B, head_dim), fill, dtype=dtype, device=device)
+    v_pool = torch.full_like(k_pool, fill)
+
+    def write(slots, kt, vt):
+        s = np.asarray(slots, np.int64)
+        ph = torch.as_tensor(s // B, device=device)
+        sl = torch.as_tensor(s % B, device=device)
+        k_pool[ph, :, sl, :] = kt
+        v_pool[ph, :, sl, :] = vt
+
+    def copy(copies):
+        if copies:
+            src = torch.as_tensor([c.src for c in copies], device=device)
+            dst = torch.as_tensor([c.dst for c in copies], device=device)
+            k_pool[dst] = k_pool[src]
+            v_pool[dst] = v_pool[src]
+
+    searches = []
+    for _ in range(num_requests):
+        bs = BeamSearch(alloc, prompt_len, width)
+        t = np.arange(prompt_len)
+        write(np.asarray(bs.beams[0].table)[t // B] * B + t % B,
+              _randn((prompt_len, num_kv_heads, head_dim), gen, dtype, device),
+              _randn((prompt_len, num_kv_heads, head_dim), gen, dtype, device))
+        searches.append(bs)
+
+    def one_step():
+        slots, copies = [], []
+        for bs in searches:
+            s, c = bs.step(rng.integers(0, width, size=width))
+            slots += s
+            copies += c
+        copy(copies)
+        return slots, len(copies)
+
+    for _ in range(steps):
+        slots, _ = one_step()
+        n = len(slots)
+        write(slots, _randn((n, num_kv_heads, head_dim), gen, dtype, device),
+              _randn((n, num_kv_heads, head_dim), gen, dtype, device))
+    slots, ncopies = one_step()
+    beams = [b for bs in searches for b in bs.beams]
+    S = len(beams)
+    max_nb = max(len(b.table) for b in beams)
+    bt = np.full((S, max_nb), -1, dtype=np.int32)
+    for i, b in enumerate(beams):
+        bt[i, :len(b.table)] = b.table
+    q = _randn((S, num_heads, head_dim), gen, dtype, device)
+    k_new = _randn((S, num_kv_heads, head_dim), gen, dtype, device)
+    v_new = _randn((S, num_kv_heads, head_dim), gen, dtype, device)
+    in_use = sum(bs.blocks_in_use() for bs in searches)
+    unshared = sum(bs.blocks_unshared() for bs in searches)
+    return DecodeCase(
+        name="beam_search", q=q, k_pool=k_pool, v_pool=v_pool,
+        block_tables=torch.as_tensor(bt, device=device),
+        context_lens=torch.as_tensor(np.asarray([b.num_tokens for b in beams], np.int32),
+                                     device=device),
+        num_heads=num_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
+        scale=1.0 / math.sqrt(head_dim), partition_size=partition_size, k_new=k_new,
+        v_new=v_new, slot_mapping=torch.as_tensor(np.asarray(slots, np.int64), device=device),
+        meta={"seed": seed, "pool_blocks": P, "requests": num_requests, "width": width,
+              "blocks_in_use": in_use, "blocks_unshared": unshared,
+              "copies_last_step": ncopies, "allocator": alloc, "searches": searches})

@@ -184,3 +184,44 @@ def test_adopt_takes_over_existing_tables():
     assert gpu.refcount(5) == 2 and other.table == [5]
     with pytest.raises(ValueError):
         gpu.adopt([1], 40)  # 40 tokens need 3 blocks
+
+
+# ---------------------------------------------------------------------------
+# beam search (page "PagedAttention Analysis", section 4): beams share the
+# prompt and intermediate blocks; the sharing pattern changes every step
+# ---------------------------------------------------------------------------
+
+from pkv_inputs import BeamSearch  # noqa: E402
+
+
+def test_beam_search_sharing_and_no_leaks():
+    B, W = 16, 4
+    alloc = BlockAllocator(200, B)
+    bs = BeamSearch(alloc, prompt_tokens=40, width=W)
+    rng = np.random.default_rng(3)
+    for t in range(60):
+        parents = rng.integers(0, W, size=W) if t % 7 else np.zeros(W, dtype=int)
+        slots, copies = bs.step(parents)
+        assert len(slots) == W and len(set(slots)) == W  # every beam writes its own slot
+        for b in bs.beams:
+            assert alloc.refcount(b.table[-1]) == 1  # the block being written is private
+        # every block of a beam is referenced at least once per beam that holds it
+        for blk in {x for b in bs.beams for x in b.table}:
+            assert alloc.refcount(blk) == sum(b.table.count(blk) for b in bs.beams)
+        assert bs.blocks_in_use() <= bs.blocks_unshared()
+    bs.release()
+    assert alloc.num_free == 200
+
+
+def test_beam_search_all_continue_one_parent_shares_everything_but_the_last_block():
+    B, W = 16, 4
+    alloc = BlockAllocator(100, B)
+    bs = BeamSearch(alloc, prompt_tokens=32, width=W)  # two full prompt blocks
+    for _ in range(20):
+        bs.step([0] * W)
+    # 52 tokens: 3 full blocks + 4 tokens; the beams share the blocks beam 0
+    # held, and each has its own last block
+    tables = [b.table for b in bs.beams]
+    assert all(t[:-1] == tables[0][:-1] for t in tables)
+    assert len({t[-1] for t in tables}) == W
+    assert bs.blocks_in_use() == len(tables[0]) - 1 + W
