@@ -351,7 +351,11 @@ def config_block(case, workload, n_gpus):
                 "(the timed step is the 64th)" if workload == "shared_prefix" else
         "beam search: 32 requests x 4 beams, 32 q heads / 8 kv heads, head_dim 128, bf16, "
         "block 16, prompt 512, seeded random parents each step; the timed step is the 128th "
-        "(append + decode of the 128 beams)" if workload == "beam_search" else workload)
+        "(append + decode of the 128 beams)" if workload == "beam_search" else
+        "automatic prefix caching: 64 requests, 1024-token system prompt shared by all, 8 "
+        "groups sharing a 512-token prefix, unique 128-256-token suffixes; 32 q / 8 kv heads, "
+        "head_dim 128, bf16, block 16; blocks keyed by a hash of the whole prefix"
+        if workload == "prefix_cache" else workload)
     return {
         "workload": workload, "desc": desc, "num_seqs_per_gpu": case.num_seqs,
         "num_heads": case.num_heads, "num_kv_heads": case.num_kv_heads,
@@ -394,6 +398,24 @@ def build_bench_case(args, dev, rank):
             "note": "value/roofline count logical bytes; blocks shared by the beams of a "
                     "request are read from L2"}}
         case.meta = {k: v for k, v in m.items() if k not in ("allocator", "searches")}
+        return case, extras
+    if args.workload == "prefix_cache":
+        # 64 requests: a 1024-token system prompt shared by all, 8 groups sharing a
+        # 512-token prefix, unique 128-256-token suffixes; blocks from the prefix
+        # cache; the timed step appends each request's last token and decodes.
+        from pkv_inputs import make_prefix_cache_case
+        case = make_prefix_cache_case(device=dev, seed=rank_seed(394, rank))
+        m = case.meta
+        per_tok = 2 * case.num_kv_heads * case.head_dim * case.k_pool.element_size()
+        extras = {"prefix_cache": {
+            "hits": m["hits"], "misses": m["misses"],
+            "blocks_in_use": m["blocks_in_use"], "blocks_unshared": m["blocks_unshared"],
+            "memory_saving": 1.0 - m["blocks_in_use"] / m["blocks_unshared"],
+            "logical_kv_bytes": int(case.context_lens.sum()) * per_tok,
+            "unique_kv_bytes": m["blocks_in_use"] * per_tok * case.block_size,
+            "note": "value/roofline count logical bytes; cached prefix blocks are read "
+                    "from L2 by the requests that share them"}}
+        case.meta = {k: v for k, v in m.items() if k not in ("cache", "tokens")}
         return case, extras
     if args.workload != "shared_prefix":
         case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
@@ -750,9 +772,10 @@ def run_ours(args, rank, world, local_rank):
     line["config"]["call"] = ("kv_cache_append + paged_attn_decode" if not fused else
                               "paged_attn_decode_append (append fused into the decode)")
     line.update(extras)
-    if "beam_search" in extras:
-        bx = extras["beam_search"]
-        bx["unique_gbs"] = bx["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
+    for key in ("beam_search", "prefix_cache"):
+        if key in extras:
+            bx = extras[key]
+            bx["unique_gbs"] = bx["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
     if "shared_prefix" in extras:
         sp_x = extras["shared_prefix"]
         sp_x["unique_gbs"] = sp_x["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9

@@ -17,9 +17,9 @@ Modules:
 """
 
 from .block_manager import (  # noqa: F401
-    BeamSearch, BlockAllocator, BlockMove, CowCopy, SeqState, SwapSpace)
+    BeamSearch, BlockAllocator, BlockMove, CowCopy, PrefixCache, SeqState, SwapSpace)
 from .workloads import (  # noqa: F401
-    make_beam_search_case,
+    make_beam_search_case, make_prefix_cache_case,
     DecodeCase,
     POOL_LAYOUT,
     WORKLOADS,

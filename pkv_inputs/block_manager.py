@@ -35,6 +35,7 @@ memory, which matches the pages' point that block management needs no
 
 from __future__ import annotations
 
+import hashlib
 from collections import Counter
 from dataclasses import dataclass, field
 from typing import List, Optional, Sequence, Tuple
@@ -112,12 +113,18 @@ class BlockAllocator:
         self._ref[b] = 1
         return b
 
-    def free(self, block: int) -> None:
+    def free(self, block: int, reuse_last: bool = False) -> None:
+        """Drop one reference. A block nobody references goes back to the free
+        list: next in line to be handed out, or with ``reuse_last`` at the back
+        of the line (a cached block that should survive as long as possible)."""
         if self._ref[block] <= 0:
             raise ValueError(f"block {block} freed more often than referenced")
         self._ref[block] -= 1
         if self._ref[block] == 0:
-            self._free.append(block)
+            if reuse_last:
+                self._free.insert(0, block)
+            else:
+                self._free.append(block)
 
     def reference(self, block: int) -> None:
         """Add a reference to a block, taking it off the free list if it was free."""
@@ -287,3 +294,74 @@ class BeamSearch:
         for b in self.beams:
             self.alloc.release(b)
         self.beams = []
+
+
+class PrefixCache:
+    """Automatic prefix caching over a BlockAllocator (page "PagedAttention
+    Analysis", ryotta.opik.net, section 4: each KV block is identified by a
+    hash of the prefix tokens and registered in a global hash table, so common
+    prefixes are shared without a tree).
+
+    A full block's key is a hash of every token up to and including it (the
+    previous block's key chained with this block's tokens): two sequences map a
+    block to the same physical block exactly when their whole prefixes agree up
+    to its end. A hit references the cached block; a miss allocates one, which
+    the caller must fill, and registers it. A partial last block is always
+    private and never cached. A released cached block keeps its contents and its
+    key until the allocator hands it out again: it goes to the back of the free
+    list, behind every block that holds nothing, and of one released prefix the
+    later blocks go before the earlier ones.
+    """
+
+    def __init__(self, alloc: BlockAllocator):
+        self.alloc = alloc
+        self.table: dict = {}     # prefix key -> physical block
+        self.key_of: dict = {}    # physical block -> prefix key
+        self.hits = 0
+        self.misses = 0
+
+    @staticmethod
+    def block_keys(tokens: Sequence[int], block_size: int) -> List[bytes]:
+        keys, prev = [], b""
+        for j in range(len(tokens) // block_size):
+            blk = np.asarray(tokens[j * block_size:(j + 1) * block_size], dtype=np.int64)
+            prev = hashlib.blake2b(prev + blk.tobytes(), digest_size=16).digest()
+            keys.append(prev)
+        return keys
+
+    def _allocate(self) -> int:
+        b = self.alloc.allocate()
+        k = self.key_of.pop(b, None)
+        if k is not None:  # evicted: its contents are about to be overwritten
+            del self.table[k]
+        return b
+
+    def new_sequence(self, tokens: Sequence[int]) -> Tuple[SeqState, List[int]]:
+        """The sequence's block table, and the logical blocks the caller must fill
+        (the misses and the partial last block)."""
+        B = self.alloc.block_size
+        table, fills = [], []
+        for j, k in enumerate(self.block_keys(tokens, B)):
+            b = self.table.get(k)
+            if b is not None:
+                self.alloc.reference(b)
+                self.hits += 1
+            else:
+                b = self._allocate()
+                self.table[k] = b
+                self.key_of[b] = k
+                fills.append(j)
+                self.misses += 1
+            table.append(b)
+        if len(tokens) % B:
+            table.append(self._allocate())
+            fills.append(len(table) - 1)
+        return SeqState(table=table, num_tokens=len(tokens)), fills
+
+    def release(self, seq: SeqState) -> None:
+        # last block first: of a released prefix, the later blocks are evicted
+        # before the earlier ones (a later key is useless without the earlier)
+        for b in reversed(seq.table):
+            self.alloc.free(b, reuse_last=b in self.key_of)
+        seq.table = []
+        seq.num_tokens = 0

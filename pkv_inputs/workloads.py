@@ -32,7 +32,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 import torch
 
-from .block_manager import BeamSearch, BlockAllocator
+from .block_manager import BeamSearch, BlockAllocator, PrefixCache
 
 POOL_LAYOUT = "[num_blocks][num_kv_heads][block_size][head_dim], head_dim contiguous"
 
@@ -486,3 +486,71 @@ def make_beam_search_case(device="cpu", seed: int = 393, num_requests: int = 32,
         meta={"seed": seed, "pool_blocks": P, "requests": num_requests, "width": width,
               "blocks_in_use": in_use, "blocks_unshared": unshared,
               "copies_last_step": ncopies, "allocator": alloc, "searches": searches})
+
+
+def make_prefix_cache_case(device="cpu", seed: int = 394, num_requests: int = 64,
+                           system_len: int = 1024, groups: int = 8, group_len: int = 512,
+                           suffix_range=(128, 256), num_heads: int = 32, num_kv_heads: int = 8,
+                           head_dim: int = 128, block_size: int = 16, dtype=torch.bfloat16,
+                           partition_size: int = DEFAULT_PARTITION):
+    """Automatic prefix caching (page "PagedAttention Analysis", section 4):
+    requests built from synthetic token ids (a system prompt shared by all, a
+    prefix shared within each of ``groups`` groups, a unique suffix) get their
+    blocks from a PrefixCache. Each block that misses the cache is filled with
+    N(0,1) K/V when it is first allocated; hits read what was written then.
+    The total length of a request is never a multiple of the block size, and its
+    last token is the one the step appends (``k_new``/``v_new``/``slot_mapping``),
+    so the appended token always lands in the request's private last block.
+    Cache statistics are in ``meta``."""
+    B = block_size
+    rng = np.random.default_rng(seed)
+    gen = _generator(seed, device)
+    system = rng.integers(0, 32000, size=system_len).tolist()
+    group_prefix = [rng.integers(0, 32000, size=group_len).tolist() for _ in range(groups)]
+    reqs = []
+    for r in range(num_requests):
+        n = int(rng.integers(suffix_range[0], suffix_range[1] + 1))
+        total = system_len + group_len + n
+        if total % B == 0:
+            n += 1
+        reqs.append(system + group_prefix[r % groups] + rng.integers(0, 32000, size=n).tolist())
+    P = sum(-(-len(t) // B) for t in reqs)  # enough without any sharing
+    alloc = BlockAllocator(P, B, free_order=rng.permutation(P).tolist())
+    cache = PrefixCache(alloc)
+    fill = float("nan")
+    k_pool = torch.full((P, num_kv_heads, B, head_dim), fill, dtype=dtype, device=device)
+    v_pool = torch.full_like(k_pool, fill)
+    seqs = []
+    for toks in reqs:
+        sq, fills = cache.new_sequence(toks)
+        L = len(toks)
+        for j in fills:
+            n = min(B, L - 1 - j * B)  # the last token is appended by the step itself
+            if n <= 0:
+                continue
+            blk = sq.table[j]
+            k_pool[blk, :, :n, :] = _randn((num_kv_heads, n, head_dim), gen, dtype, device)
+            v_pool[blk, :, :n, :] = _randn((num_kv_heads, n, head_dim), gen, dtype, device)
+        seqs.append(sq)
+    S = len(seqs)
+    max_nb = max(len(sq.table) for sq in seqs)
+    bt = np.full((S, max_nb), -1, dtype=np.int32)
+    for i, sq in enumerate(seqs):
+        bt[i, :len(sq.table)] = sq.table
+    lens = np.asarray([sq.num_tokens for sq in seqs], np.int32)
+    slots = np.asarray([sq.table[(L - 1) // B] * B + (L - 1) % B for sq, L in zip(seqs, lens)],
+                       np.int64)
+    q = _randn((S, num_heads, head_dim), gen, dtype, device)
+    k_new = _randn((S, num_kv_heads, head_dim), gen, dtype, device)
+    v_new = _randn((S, num_kv_heads, head_dim), gen, dtype, device)
+    in_use = len({b for sq in seqs for b in sq.table})
+    return DecodeCase(
+        name="prefix_cache", q=q, k_pool=k_pool, v_pool=v_pool,
+        block_tables=torch.as_tensor(bt, device=device),
+        context_lens=torch.as_tensor(lens, device=device),
+        num_heads=num_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
+        scale=1.0 / math.sqrt(head_dim), partition_size=partition_size, k_new=k_new,
+        v_new=v_new, slot_mapping=torch.as_tensor(slots, device=device),
+        meta={"seed": seed, "pool_blocks": P, "hits": cache.hits, "misses": cache.misses,
+              "blocks_in_use": in_use, "blocks_unshared": int(sum(len(sq.table) for sq in seqs)),
+              "tokens": [list(t) for t in reqs], "cache": cache})

@@ -225,3 +225,64 @@ def test_beam_search_all_continue_one_parent_shares_everything_but_the_last_bloc
     assert all(t[:-1] == tables[0][:-1] for t in tables)
     assert len({t[-1] for t in tables}) == W
     assert bs.blocks_in_use() == len(tables[0]) - 1 + W
+
+
+# ---------------------------------------------------------------------------
+# automatic prefix caching (page "PagedAttention Analysis", section 4): blocks
+# keyed by a hash of the whole prefix, shared through a global table
+# ---------------------------------------------------------------------------
+
+from pkv_inputs import PrefixCache  # noqa: E402
+
+
+def test_prefix_keys_chain_the_whole_prefix():
+    B = 16
+    a = list(range(100))
+    b = a[:32] + [7] * 68
+    c = [999] + a[1:]
+    ka, kb, kc = (PrefixCache.block_keys(t, B) for t in (a, b, c))
+    assert len(ka) == 6  # full blocks only
+    assert ka[:2] == kb[:2] and ka[2] != kb[2]
+    assert all(x != y for x, y in zip(ka, kc))  # a change in block 0 changes every key
+
+
+def test_prefix_cache_hits_misses_and_private_tails():
+    B = 16
+    pc = PrefixCache(BlockAllocator(64, B))
+    sys_prompt = list(range(1000, 1064))  # 4 full blocks
+    a, fa = pc.new_sequence(sys_prompt + list(range(40)))
+    assert (pc.hits, pc.misses) == (0, 6) and fa == [0, 1, 2, 3, 4, 5, 6]
+    b, fb = pc.new_sequence(sys_prompt + list(range(500, 540)))
+    assert pc.hits == 4 and b.table[:4] == a.table[:4]
+    assert fb == [4, 5, 6] and not set(b.table[4:]) & set(a.table)
+    c, fc = pc.new_sequence(sys_prompt + list(range(40)))  # same tokens as a
+    assert c.table[:6] == a.table[:6] and c.table[6] != a.table[6]  # the partial block is private
+    assert fc == [6]
+    assert pc.alloc.refcount(a.table[0]) == 3
+
+
+def test_prefix_cache_survives_release_and_evicts_cleanly():
+    B = 16
+    alloc = BlockAllocator(12, B)
+    pc = PrefixCache(alloc)
+    toks = list(range(64))
+    a, _ = pc.new_sequence(toks)
+    a_table = list(a.table)
+    pc.release(a)
+    assert alloc.num_free == 12 and len(pc.table) == 4  # still cached
+    b, fills = pc.new_sequence(toks)
+    assert fills == [] and b.table == a_table  # all four blocks hit
+    assert pc.hits == 4
+    pc.release(b)
+    # unrelated requests take the 8 empty blocks first, then evict cached
+    # blocks, the prefix's last ones first; an evicted block leaves the table
+    others = [pc.new_sequence([5000 + 100 * i + t for t in range(32)])[0] for i in range(5)]
+    assert len(pc.table) == 2 + 10
+    for k, blk in pc.table.items():
+        assert pc.key_of[blk] == k
+    for sq in others:
+        pc.release(sq)
+    c, fills = pc.new_sequence(toks)
+    assert c.table[:2] == a_table[:2] and fills == [2, 3]  # blocks 0, 1 survived
+    pc.release(c)
+    assert alloc.num_free == 12
