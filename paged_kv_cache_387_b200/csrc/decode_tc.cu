@@ -308,6 +308,13 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Add `bytes` to the current phase's expected transaction count, without an
+// arrival (the phase completes after the arrivals and all the bytes).
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
 // Bulk copy global -> shared (no tensor map), completing on an mbarrier.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
                                           uint32_t bar) {
@@ -546,30 +553,16 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int t_begin = p * a.part_tokens;
       const int t_end = min(L, t_begin + a.part_tokens);
       const int n_tiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
-      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
-      constexpr int upt = U8 ? 2 : 1;  // table entries per tile
-      for (int t = lane; t < n_tiles * upt && t < DESC_IDS; t += 32) {
-        const int tok = t_begin + t * (TILE / upt);
-        d.ids[t] = tok < L ? bt[tok / B] : -1;  // no table entry is read past the context
-      }
       // Fused append: the partition holding token L-1 also stages that
       // token's new K and V rows.
       const bool has_new = a.k_new != nullptr && n_tiles > 0 && t_end == L;
-      if (lane == 0) {
-        d.kind = KIND_WORK;
-        d.s = s;
-        d.p = p;
-        d.h = h;
-        d.L = L;
-        d.n_tiles = n_tiles;
-        d.nparts = (L + a.part_tokens - 1) / a.part_tokens;
-        d.new_tok = has_new ? L - 1 - t_begin : -1;
-      }
-      __syncwarp();  // every lane's ids precede lane 0's release below
+      // The group's q rows (and the new rows) are copied first: the copies
+      // complete on the slot's barrier while the lanes fetch the block ids,
+      // and the arrival that publishes the descriptor comes last.
       if (lane == 0) {
         const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
         const uint32_t rbytes = has_new ? (uint32_t)(D * 2) : 0u;
-        mbar_arrive_expect_tx(item_full(slot), qbytes + 2 * rbytes);
+        mbar_expect_tx(item_full(slot), qbytes + 2 * rbytes);
         const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES;
         if (qbytes)
           bulk_load(stage, static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
@@ -582,6 +575,24 @@ __global__ void __launch_bounds__(THREADS, 2)
                     rbytes, item_full(slot));
         }
       }
+      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
+      constexpr int upt = U8 ? 2 : 1;  // table entries per tile
+      for (int t = lane; t < n_tiles * upt && t < DESC_IDS; t += 32) {
+        const int tok = t_begin + t * (TILE / upt);
+        d.ids[t] = tok < L ? bt[tok / B] : -1;  // no table entry is read past the context
+      }
+      if (lane == 0) {
+        d.kind = KIND_WORK;
+        d.s = s;
+        d.p = p;
+        d.h = h;
+        d.L = L;
+        d.n_tiles = n_tiles;
+        d.nparts = (L + a.part_tokens - 1) / a.part_tokens;
+        d.new_tok = has_new ? L - 1 - t_begin : -1;
+      }
+      __syncwarp();  // every lane's ids precede lane 0's release below
+      if (lane == 0) mbar_arrive(item_full(slot));
       ++in_flight;
       if (prefetch)
         item = __shfl_sync(FULL_MASK, next, 0);

@@ -263,3 +263,27 @@ def test_decode_accuracy_short_contexts_with_cancellation(dt, seed):
     for part in (0, 16):
         got = gpu_decode(c, partition_size=part)
         assert_close_to_oracle(got, oracle_decode(c), DT[dt], f"short {dt} s{seed} p{part}")
+
+
+@pytest.mark.parametrize("dt,B,part", [(torch.bfloat16, 16, 0), (torch.float16, 8, 32)])
+def test_many_short_sequences(dt, B, part):
+    """Thousands of sequences (the plan takes them in many rounds; contexts of 0
+    to 80 tokens; with 32-token partitions many are split), every output
+    checked against the oracle."""
+    lens = np.random.default_rng(13).integers(0, 81, size=3000).tolist()
+    c = make_random_case("many", 8, 2, 64, B, lens, dt, seed=29, device=DEV)
+    err = new_err(DEV)
+    got = gpu_decode(c, partition_size=part, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert_close_to_oracle(got, oracle_decode(c), dt, f"3000 seqs B{B} p{part}")
+
+
+def test_max_group_and_block_size():
+    """The largest supported group (8 query heads per KV head) with the largest
+    block size (256 tokens), contexts spanning several blocks and partitions."""
+    c = make_random_case("maxgb", 32, 4, 128, 256, [1, 255, 256, 257, 1500, 3000], torch.bfloat16,
+                         seed=31, device=DEV)
+    for part in (0, 256, 1024):
+        assert_close_to_oracle(gpu_decode(c, partition_size=part), oracle_decode(c),
+                               torch.bfloat16, f"G8 B256 p{part}")
