@@ -277,6 +277,20 @@ int kv_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v
                   int block_size, int src_blocks, int dst_blocks, int dtype, int32_t *err,
                   void *stream);
 
+/*
+ * pkv_check_wait_timeout - diagnostic of the bounded waits. Every wait of the
+ * decode kernels on an mbarrier gives up after about a second, stores
+ * PKV_DEV_WAIT_TIMEOUT in *err and winds the kernel down instead of hanging.
+ * This call runs that same wait on a barrier phase that nothing completes,
+ * with a limit of limit_cycles SM clock cycles (1 .. 4e9), so the give-up path
+ * can be exercised without any fault. err is a device pointer (not NULL); it
+ * receives PKV_DEV_WAIT_TIMEOUT if it held 0. The kernel then returns and the
+ * context stays usable. An fp16/bf16 decode called while *err holds
+ * PKV_DEV_WAIT_TIMEOUT does no work (its output and the pools are left as they
+ * were): the caller resets *err to 0 first. The fp32 path has no such waits.
+ */
+int pkv_check_wait_timeout(long long limit_cycles, int32_t *err, void *stream);
+
 /* Static, human-readable text for a pkv_status value. */
 const char *pkv_status_string(int status);
 

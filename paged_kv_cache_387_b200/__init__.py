@@ -30,7 +30,8 @@ DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 DEFAULT_PARTITION = 2048  # tokens per split-context partition (measured best on B200)
 
 EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
-           "kv_block_copy", "kv_block_swap", "pkv_decode_workspace_bytes", "pkv_status_string")
+           "kv_block_copy", "kv_block_swap", "pkv_check_wait_timeout",
+           "pkv_decode_workspace_bytes", "pkv_status_string")
 
 
 class PkvError(RuntimeError):
@@ -64,6 +65,8 @@ def load_library():
     lib.kv_block_copy.restype = I
     lib.kv_block_swap.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P]
     lib.kv_block_swap.restype = I
+    lib.pkv_check_wait_timeout.argtypes = [ctypes.c_longlong, P, P]
+    lib.pkv_check_wait_timeout.restype = I
     lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_bytes.restype = Z
     lib.pkv_status_string.argtypes = [I]
@@ -272,6 +275,15 @@ def kv_block_swap(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
                            D, B, Ps, Pd, DTYPE_CODES[dt], _dev_ptr(err, "err", device),
                            _stream_ptr(stream, device))
     _check("kv_block_swap", rc)
+
+
+def check_wait_timeout(err: torch.Tensor, limit_cycles: int = 2_000_000, stream=None) -> None:
+    """Run the decode kernels' bounded wait on a barrier nothing completes; the
+    wait gives up after ``limit_cycles`` and stores PKV_DEV_WAIT_TIMEOUT in err."""
+    lib = load_library()
+    rc = lib.pkv_check_wait_timeout(int(limit_cycles), _dev_ptr(err, "err", err.device),
+                                    _stream_ptr(stream, err.device))
+    _check("pkv_check_wait_timeout", rc)
 
 
 def device_error_message(code: int) -> str:

@@ -304,6 +304,13 @@ int kv_block_copy(void *k_pool, void *v_pool, const int32_t *src_dst, int num_pa
                                             num_blocks, err, static_cast<cudaStream_t>(stream)));
 }
 
+int pkv_check_wait_timeout(long long limit_cycles, int32_t *err, void *stream) {
+  if (limit_cycles <= 0 || limit_cycles > 4000000000LL || !err || !aligned(err, 4))
+    return PKV_EINVAL;
+  return cuda_status(pkv::launch_wait_timeout_probe(limit_cycles, err,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
 int kv_block_swap(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
                   const int32_t *src_dst, int num_pairs, int num_kv_heads, int head_dim,
                   int block_size, int src_blocks, int dst_blocks, int dtype, int32_t *err,

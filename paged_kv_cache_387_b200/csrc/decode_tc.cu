@@ -275,18 +275,37 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
 // case it sets the flag and reports PKV_DEV_WAIT_TIMEOUT. Either way the
 // caller leaves its loop, so a failure ends the kernel instead of stalling.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
-                                              volatile int *abort_flag, int32_t *err) {
+                                              volatile int *abort_flag, int32_t *err,
+                                              long long limit = WAIT_LIMIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       report(err, PKV_DEV_WAIT_TIMEOUT);
       return false;
     }
   }
   return true;
+}
+
+// Diagnostic: one block waits, through wait_or_abort, on an mbarrier phase
+// that nothing completes, with a short limit. The wait must give up, set the
+// abort flag and report PKV_DEV_WAIT_TIMEOUT, and the kernel must return; the
+// decode kernels' waits run the same code with the long limit.
+__global__ void wait_timeout_probe_kernel(long long limit, int32_t *err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);  // one arrival expected; none ever comes
+    fence_mbar_init();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  const bool ok = wait_or_abort(b, 0, &abort_flag, err, limit);
+  if (ok && threadIdx.x == 0) report(err, PKV_DEV_BAD_PAIR);  // a phase completed: wrong
 }
 
 // Non-blocking test of an mbarrier phase.
@@ -439,22 +458,23 @@ __global__ void __launch_bounds__(THREADS, 2)
     fence_mbar_init();
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
-  }
-  pdl_wait();  // the work list, counters and everything before the plan are ready
-  if (threadIdx.x == 0) {
-    // A CTA that starts after some wait already gave up does no work.
-    s_abort = (a.err != nullptr &&
-               *reinterpret_cast<volatile const int32_t *>(a.err) == PKV_DEV_WAIT_TIMEOUT)
-                  ? 1
-                  : 0;
+    s_abort = 0;
   }
   __syncthreads();
+  pdl_wait();  // the work list, counters and everything before the plan are ready
 
   if (warp == NCW) {
     // ======================= scheduler warp =======================
     const long long list_cap = (long long)a.num_seqs * a.max_parts;
     const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
     const int end_phase = total_items - END_ITEMS_PER_CTA * (int)gridDim.x;
+    // A CTA that starts after some wait already gave up does no work. The
+    // error word is loaded now and checked before the first copy is started,
+    // so its latency overlaps the first work-list load.
+    const int32_t err_word = (lane == 0 && a.err != nullptr)
+                                 ? *reinterpret_cast<volatile const int32_t *>(a.err)
+                                 : 0;
+    bool first_post = true;
     int item = blockIdx.x;  // the first item of every CTA is fixed; the counter starts at grid
     bool claimed = true;  // `item` holds an index taken from the work list
     int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
@@ -556,6 +576,13 @@ __global__ void __launch_bounds__(THREADS, 2)
       // Fused append: the partition holding token L-1 also stages that
       // token's new K and V rows.
       const bool has_new = a.k_new != nullptr && n_tiles > 0 && t_end == L;
+      if (first_post) {
+        first_post = false;
+        if (__shfl_sync(FULL_MASK, err_word == PKV_DEV_WAIT_TIMEOUT ? 1 : 0, 0)) {
+          if (lane == 0) *abort_flag = 1;  // the consumers' waits see it and stop
+          break;
+        }
+      }
       // The group's q rows (and the new rows) are copied first: the copies
       // complete on the slot's barrier while the lanes fetch the block ids,
       // and the arrival that publishes the descriptor comes last.
@@ -1044,6 +1071,11 @@ cudaError_t launch_tc_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUten
 
 size_t decode_tc_smem_bytes(int head_dim) {
   return head_dim == 64 ? TcShape<64, 8>::SMEM_BYTES : TcShape<128, 8>::SMEM_BYTES;
+}
+
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, int32_t *err, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(limit_cycles, err);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,

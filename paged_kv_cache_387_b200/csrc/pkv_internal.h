@@ -61,6 +61,7 @@ struct WorkspaceLayout {
 WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long long max_parts);
 
 // Plan + persistent decode (+ merge when split) for fp16 / bf16.
+cudaError_t launch_wait_timeout_probe(long long limit_cycles, int32_t *err, cudaStream_t stream);
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t stream);
 cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream);

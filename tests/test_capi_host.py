@@ -122,3 +122,10 @@ def test_binding_refuses_unpinned_host_output(lib):
     bt = torch.zeros(2, 1, dtype=torch.int32)
     with pytest.raises(ValueError, match="pinned"):
         pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
+
+
+def test_wait_timeout_check_arguments(lib):
+    f = lib.pkv_check_wait_timeout
+    assert f(0, FAKE, None) == pkv.PKV_EINVAL           # limit must be positive
+    assert f(5_000_000_000, FAKE, None) == pkv.PKV_EINVAL
+    assert f(1000, None, None) == pkv.PKV_EINVAL         # err is required
