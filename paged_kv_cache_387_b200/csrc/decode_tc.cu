@@ -13,26 +13,37 @@
 //
 // Scheduling
 //   A one-CTA plan kernel turns context_lens into a compact work list of
-//   (sequence, partition) pairs: full partitions first, then the shorter last
-//   partitions. It also resets the dispatch and merge counters. The decode
-//   kernel is persistent, two CTAs per SM, and pulls items (pair x KV head)
-//   from an atomic counter until the list is exhausted. It is launched as a
-//   programmatic dependent of the plan, so its set-up overlaps the plan.
+//   (sequence, partition) pairs. Sequences of several partitions come first,
+//   each with its short last partition first. Sequences of one partition
+//   follow, largest first, with batch order kept within a size class. The plan
+//   also resets the dispatch and merge counters. The decode kernel is
+//   persistent, two CTAs per SM. Each CTA takes item blockIdx.x first, then
+//   pulls items (pair x KV head) from an atomic counter until the list is
+//   exhausted. Launches chain by programmatic dependence: the plan starts
+//   while the previous call finishes, and the decode grid's set-up overlaps
+//   the plan.
 //
 // Warp roles
-//   Warp 4 is the scheduler. It resolves items ahead of use (work-list
-//   entry, context length, the physical block id of every 16-token tile) and
-//   posts them as descriptors into a small ring, with the group's q rows
-//   fetched by one bulk copy. It also keeps the partition count. When the
-//   consumers finish an item of a split context, the scheduler publishes it
-//   (a device-scope fence and a fetch-and-add on the (sequence, KV head)
-//   counter). The CTA that completes the last partition receives a merge
-//   task in its descriptor stream. No CTA ever waits for another.
+//   Warp 4 is the scheduler. It resolves items ahead of use and posts them as
+//   descriptors into a small ring: the work-list entry (with the context
+//   length), the physical block ids of up to DESC_IDS tiles, and the group's q
+//   rows, fetched by one bulk copy. In the last few items per CTA it holds at
+//   most two descriptors, which spreads the final items over the CTAs. It
+//   also keeps the partition count. When the consumers finish an item of a
+//   split context, the scheduler publishes it (a device-scope fence and a
+//   fetch-and-add on the (sequence, KV head) counter). The CTA that completes
+//   the last partition receives a merge task in its descriptor stream. No CTA
+//   ever waits for another.
 //   Warps 0-3 are consumers. Each owns a ring of stages in shared memory and
 //   takes tiles w, w+4, w+8, ... of every item. Its lane 0 fills the ring
-//   with TMA: per tile, 2D loads of K and V (64-element boxes, 128-byte
-//   swizzle) completing on the stage's mbarrier. The fill runs ahead of the
-//   warp's math across item boundaries. No load uses cluster multicast.
+//   with TMA, completing on the stage's mbarrier:
+//     - head_dim 128: one 3D copy per pool covers both 64-element halves of a
+//       16-token tile;
+//     - head_dim 64: one 2D copy per pool;
+//     - block sizes that are odd multiples of 8: two 8-row boxes per
+//       64-element half, one per 8-token unit, each from its own block.
+//   The boxes are 128-byte swizzled. The fill runs ahead of the warp's math
+//   across item boundaries. No load uses cluster multicast.
 //
 // Math (per tile, per consumer warp), fp32 accumulation:
 //   S^T[16 tok][8] = K_tile[16][D] . Q^T[D][8]  mma.sync m16n8k16. K is the A
@@ -45,8 +56,9 @@
 //     rescaling rare. Masked tokens get -inf, and their V rows are zeroed in
 //     shared memory before they reach the tensor core.
 //   O^T[D][8] += V^T[D][16] . P^T[16][8]  V^T via ldmatrix.trans; P^T from the
-//     score fragment via movmatrix.trans. P is split into hi + lo parts in the
-//     input type, two MMAs, so the weights keep ~16 significant bits.
+//     score fragment via movmatrix.trans. For bf16, P is split into hi + lo
+//     bf16 parts (two MMAs), so the weights keep ~16 significant bits; fp16
+//     keeps one operand (11 bits).
 // At the end of an item the consumer warps' (max, sum, output) are combined in
 // shared memory. The result goes to `out` when the sequence has one
 // partition, and otherwise to the workspace as (normalised o_p,
