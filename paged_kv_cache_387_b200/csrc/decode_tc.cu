@@ -86,6 +86,7 @@ constexpr int DESC_IDS = 64;
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
 constexpr int PLAN_THREADS = 256;
+constexpr int PLAN_STAGED_ENTRIES = 8192;  // work lists up to this size are staged in shared memory
 constexpr float RESCALE_SLACK = 8.f;     // lazy max: rescale only past 2^8 growth
 
 // Descriptor kinds (in ItemDesc::kind).
@@ -153,24 +154,30 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
 // Each entry carries the sequence's clamped length. Sequences are taken in
 // rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t), so
 // that thread order is sequence order. The merge counters are reset here too.
+//
+// This grid is the programmatic dependent of what precedes it, typically the
+// previous decode call, and may start while that call is still running. Until
+// that call has completed (griddepcontrol.wait) nothing in global memory is
+// written. With `plan_staged` the list is built in shared memory before the
+// wait, from the context lengths (which nothing still running writes), and
+// only stored to the workspace after it; otherwise the plan waits first.
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
   constexpr int NW = PLAN_THREADS / 32;
+  extern __shared__ uint2 staged_list[];     // [list capacity] when a.plan_staged
   __shared__ int wsum[NW];
   __shared__ int hist[PLAN_BUCKETS];        // count, then running start of each size class
   __shared__ int wcnt[NW][PLAN_BUCKETS];    // per-warp counts of a round, then their offsets
   __shared__ int total_m_s;
+  __shared__ int total_s;
+  __shared__ int bad_len;  // a context length was clamped: reported after the wait
   pdl_launch_dependents();  // the decode grid may launch; it waits for this grid to finish
-  // This grid may itself start while the previous decode call is finishing:
-  // nothing in global memory is touched before that call has completed.
-  pdl_wait();
+  const bool staged = a.plan_staged != 0;
+  if (!staged) pdl_wait();
+  uint2 *const list = staged ? staged_list : a.work;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, P = a.part_tokens;
-  if (a.merge_cnt) {
-    const int n1 = S * a.num_kv_heads * a.max_chunks;
-    for (int i = tid; i < n1; i += PLAN_THREADS) a.merge_cnt[i] = 0;
-    for (int i = tid; i < S * a.num_kv_heads; i += PLAN_THREADS) a.merge_cnt2[i] = 0;
-  }
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
+  if (tid == 0) bad_len = 0;
   __syncthreads();
   const int max_tiles = max(1, P / 16);
   // size class of a one-partition sequence of `len` tokens: bigger -> smaller class
@@ -209,8 +216,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
     const int s = r0 + tid;
     if (s < S) {
-      const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks,
-                                  a.block_size, a.err);
+      const int raw = a.context_lens[s];
+      const int L = effective_len(raw, a.max_context_len, a.max_blocks, a.block_size, nullptr);
+      if (L < raw) bad_len = 1;
       if (L > P)
         nm += (L + P - 1) / P;
       else
@@ -231,10 +239,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     const int excl = v - h0 - h1;
     hist[2 * lane] = total_m + excl;
     hist[2 * lane + 1] = total_m + excl + h0;
-    if (lane == 31) {
-      a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
-      a.sched[1] = total_m + v;
-    }
+    if (lane == 31) total_s = total_m + v;
   }
   if (tid == 0) total_m_s = 0;
   __syncthreads();
@@ -255,8 +260,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     int round_m;
     const int om = total_m_s + block_scan(np, round_m);
     if (np > 0) {
-      a.work[om] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
-      for (int q = 0; q < np - 1; ++q) a.work[om + 1 + q] = make_uint2(pack_pair(s, q), (uint32_t)L);
+      list[om] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
+      for (int q = 0; q < np - 1; ++q) list[om + 1 + q] = make_uint2(pack_pair(s, q), (uint32_t)L);
     }
     // region 2: rank among this warp's lanes of the same class, then the
     // earlier warps' counts, then the class's running start
@@ -277,8 +282,22 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     }
     if (tid == 0) total_m_s += round_m;
     __syncthreads();
-    if (bkt >= 0) a.work[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+    if (bkt >= 0) list[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
     __syncthreads();  // wcnt and total_m_s are rewritten by the next round
+  }
+  if (staged) pdl_wait();  // the previous call has completed: the workspace is free
+  const int total = total_s;
+  if (staged)
+    for (int i = tid; i < total; i += PLAN_THREADS) a.work[i] = staged_list[i];
+  if (a.merge_cnt) {
+    const int n1 = S * a.num_kv_heads * a.max_chunks;
+    for (int i = tid; i < n1; i += PLAN_THREADS) a.merge_cnt[i] = 0;
+    for (int i = tid; i < S * a.num_kv_heads; i += PLAN_THREADS) a.merge_cnt2[i] = 0;
+  }
+  if (tid == 0) {
+    a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
+    a.sched[1] = total;
+    if (bad_len) report(a.err, PKV_DEV_CONTEXT_LEN);
   }
 }
 
@@ -1049,10 +1068,21 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // Lists that fit are built in the plan's shared memory before it waits for
+  // the previous call (see plan_kernel).
+  const long long list_cap = (long long)a.num_seqs * a.max_parts;
+  b.plan_staged = list_cap <= PLAN_STAGED_ENTRIES ? 1 : 0;
+  static bool plan_smem_set = false;
+  if (!plan_smem_set) {
+    e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PLAN_STAGED_ENTRIES * (int)sizeof(uint2));
+    if (e != cudaSuccess) return e;
+    plan_smem_set = true;
+  }
   cudaLaunchConfig_t pcfg = {};
   pcfg.gridDim = dim3(1);
   pcfg.blockDim = dim3(PLAN_THREADS);
-  pcfg.dynamicSmemBytes = 0;
+  pcfg.dynamicSmemBytes = b.plan_staged ? (size_t)list_cap * sizeof(uint2) : 0;
   pcfg.stream = stream;
   pcfg.attrs = attr;
   pcfg.numAttrs = 1;

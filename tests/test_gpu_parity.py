@@ -287,3 +287,44 @@ def test_max_group_and_block_size():
     for part in (0, 256, 1024):
         assert_close_to_oracle(gpu_decode(c, partition_size=part), oracle_decode(c),
                                torch.bfloat16, f"G8 B256 p{part}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_back_to_back_calls_with_changing_batches(fused):
+    """Consecutive calls overlap: a call's plan builds its work list while the
+    previous call is still running, and stores it once that call is done.
+    Batches of different sizes and lengths alternate on one workspace; every
+    output must equal the batch's output from a call made alone."""
+    lens_sets = [[5, 300, 1200, 40], [2100, 17, 64, 700, 33, 1000, 1], [129] * 20]
+    cases = [make_random_case(f"b2b{i}", 8, 2, 128, 16, lens, torch.bfloat16, seed=40 + i,
+                              device=DEV, with_append=fused)
+             for i, lens in enumerate(lens_sets)]
+    part = 64
+
+    def call(c, out, ws=None):
+        if fused:  # appending the same token again leaves the pool unchanged
+            pkv.paged_attn_decode_append(out, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
+                                         c.block_tables, c.context_lens, c.scale,
+                                         c.max_context_len, partition_size=part, workspace=ws)
+        else:
+            pkv.paged_attn_decode(out, c.q, c.k_pool, c.v_pool, c.block_tables, c.context_lens,
+                                  c.scale, c.max_context_len, partition_size=part, workspace=ws)
+
+    refs = []
+    for c in cases:
+        o = torch.empty_like(c.q)
+        call(c, o)
+        torch.cuda.synchronize()
+        refs.append(o)
+    need = max(pkv.decode_workspace_bytes(c.num_seqs, c.num_heads, c.head_dim,
+                                          c.max_context_len, part) for c in cases)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    outs = []
+    for i in range(45):
+        c = cases[i % 3]
+        o = torch.empty_like(c.q)
+        call(c, o, ws)
+        outs.append((i % 3, o))
+    torch.cuda.synchronize()
+    for k, o in outs:
+        assert torch.equal(o.view(torch.int16), refs[k].view(torch.int16)), f"batch {k}"
