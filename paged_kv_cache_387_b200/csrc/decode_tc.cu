@@ -80,9 +80,12 @@ constexpr int NSLOT = 3;                 // item descriptors in flight
 // items per CTA left.
 constexpr int END_ITEMS_PER_CTA = 6;
 // Block ids a descriptor carries: one per 16-token tile, or one per 8-token
-// unit when the block size is an odd multiple of 8. Further ids are read
-// from the table when their tile is fetched.
-constexpr int DESC_IDS = 64;
+// unit when the block size is an odd multiple of 8 (128 tiles cover a
+// 2048-token partition). Further ids are read from the table when their tile
+// is fetched.
+constexpr int DESC_IDS = 128;
+constexpr int IDS_PER_LANE = DESC_IDS / 32;
+static_assert(DESC_IDS % 32 == 0, "ids are fetched 32 at a time");
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
 constexpr int PLAN_THREADS = 256;
@@ -635,10 +638,17 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
       constexpr int upt = U8 ? 2 : 1;  // table entries per tile
-      for (int t = lane; t < n_tiles * upt && t < DESC_IDS; t += 32) {
+      // All of a lane's table loads are issued before its first store.
+      int idv[IDS_PER_LANE];
+#pragma unroll
+      for (int k = 0; k < IDS_PER_LANE; ++k) {
+        const int t = lane + 32 * k;
         const int tok = t_begin + t * (TILE / upt);
-        d.ids[t] = tok < L ? bt[tok / B] : -1;  // no table entry is read past the context
+        idv[k] = t < n_tiles * upt && tok < L ? bt[tok / B] : -1;  // none read past the context
       }
+#pragma unroll
+      for (int k = 0; k < IDS_PER_LANE; ++k)
+        if (lane + 32 * k < n_tiles * upt) d.ids[lane + 32 * k] = idv[k];
       if (lane == 0) {
         d.kind = KIND_WORK;
         d.s = s;
