@@ -62,8 +62,11 @@
 // At the end of an item the consumer warps' (max, sum, output) are combined in
 // shared memory. The result goes to `out` when the sequence has one
 // partition, and otherwise to the workspace as (normalised o_p,
-// log2-sum-exp). Every wait is bounded: one that gives up sets an error
-// status and a CTA-wide stop flag, and the kernel winds down.
+// log2-sum-exp). The consumers meet at two barriers per item: a vote at its
+// start (which also orders the reuse of the combine area) and one after
+// their partial rows are stored. Every wait is bounded: one that gives up
+// sets an error status and a CTA-wide stop flag, and the kernel winds down,
+// first waiting (bounded) for the copies it still has in flight.
 #include "pkv_device.cuh"
 #include "pkv_internal.h"
 
@@ -324,6 +327,17 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
   return true;
 }
 
+// Bounded wait with no abort check, for the copies still in flight when a
+// warp stops after a wait gave up: it returns once the phase completes or
+// after DRAIN_LIMIT_CYCLES, whichever is first.
+constexpr long long DRAIN_LIMIT_CYCLES = 20000000LL;
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > DRAIN_LIMIT_CYCLES) return false;
+  return true;
+}
+
 // Diagnostic: one block waits, through wait_or_abort, on an mbarrier phase
 // that nothing completes, with a short limit. The wait must give up, set the
 // abort flag and report PKV_DEV_WAIT_TIMEOUT, and the kernel must return; the
@@ -512,7 +526,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     int item = blockIdx.x;  // the first item of every CTA is fixed; the counter starts at grid
     bool claimed = true;  // `item` holds an index taken from the work list
     int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
-    for (uint32_t it = 0;; ++it) {
+    uint32_t it = 0;      // descriptors posted
+    for (;; ++it) {
       const int slot = it % NSLOT;
       ItemDesc &d = desc[slot];
       int merge_kind = -1, merge_s = 0, merge_h = 0, merge_np = 0, merge_p = 0;
@@ -667,6 +682,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       else
         claimed = false;
     }
+    // After a stop, the q copies of the last descriptors posted may still be
+    // landing in shared memory: wait for them (bounded) before leaving.
+    if (*abort_flag)
+      for (uint32_t k = it > NSLOT ? it - NSLOT : 0; k < it; ++k)
+        wait_bounded(item_full(k % NSLOT), (k / NSLOT) & 1);
     // This CTA posts nothing more: the next call's grids may start launching
     // (they wait for this grid to complete before touching memory).
     if (lane == 0) pdl_launch_dependents();
@@ -780,10 +800,14 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
   };
 
+  bool stop = false;  // a wait of this warp gave up during the previous item
   for (uint32_t it = 0;; ++it) {
     const int slot = it % NSLOT;
     const bool got = wait_or_abort(item_full(slot), (it / NSLOT) & 1, abort_flag, a.err);
-    if (!consumers_all(got)) break;
+    // One vote per item. All consumers have finished the previous item (its
+    // combine-area reads included) before any passes, and all take the same
+    // exit decision.
+    if (!consumers_all(got && !stop && *abort_flag == 0)) break;
     const ItemDesc &dref = desc[slot];
     const int kind = dref.kind;
     if (kind == KIND_END) break;  // the same descriptor for every consumer: a uniform exit
@@ -1034,13 +1058,19 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (dd == 0) a.ws_lse[row * a.max_parts + p] = scales[NH * NCW + n];
       }
     }
-    // Everyone is done with the combine area and this item's descriptor/q;
-    // the vote makes a stop (after a wait gave up anywhere) uniform. Handing
-    // the slot back also publishes this item's global writes to the scheduler.
-    const bool go_on = consumers_all(!aborted && *abort_flag == 0);
+    // This warp is done with the item's descriptor and q rows. Its arrival
+    // (after the warp's lanes have synchronised) hands the slot back and
+    // publishes the warp's global writes to the scheduler.
+    __syncwarp();
     if (lane == 0) mbar_arrive(item_empty(slot));
-    if (!go_on) break;
+    stop = aborted;
   }
+
+  // After a stop, copies this warp issued may still be landing in its ring:
+  // wait for them (bounded) before the CTA's shared memory is released.
+  for (; done != issued; ++done)
+    if (!__all_sync(FULL_MASK, wait_bounded(tile_full(warp, done % NSTAGE), (done / NSTAGE) & 1)))
+      break;
 }
 
 int sm_count_for_current_device() {
