@@ -62,9 +62,9 @@
 // At the end of an item the consumer warps' (max, sum, output) are combined in
 // shared memory. The result goes to `out` when the sequence has one
 // partition, and otherwise to the workspace as (normalised o_p,
-// log2-sum-exp). The consumers meet at two barriers per item: a vote at its
-// start (which also orders the reuse of the combine area) and one after
-// their partial rows are stored. Every wait is bounded: one that gives up
+// log2-sum-exp). The consumers meet at three barriers per item: a vote at
+// its start (which also orders the reuse of the combine area), one after
+// their partial rows are stored and one after the per-warp weights are. Every wait is bounded: one that gives up
 // sets an error status and a CTA-wide stop flag, and the kernel winds down,
 // first waiting (bounded) for the copies it still has in flight.
 #include "pkv_device.cuh"
