@@ -92,7 +92,6 @@ static_assert(DESC_IDS % 32 == 0, "ids are fetched 32 at a time");
 constexpr int BOX_COLS = 64;             // elements per TMA box row (128 bytes)
 constexpr int HALF_BYTES = TILE * 128;   // one box: 16 rows x 128 bytes
 constexpr int PLAN_THREADS = 256;
-constexpr int PLAN_STAGED_ENTRIES = 8192;  // work lists up to this size are staged in shared memory
 constexpr float RESCALE_SLACK = 8.f;     // lazy max: rescale only past 2^8 growth
 
 // Descriptor kinds (in ItemDesc::kind).
@@ -162,14 +161,12 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
 // that thread order is sequence order. The merge counters are reset here too.
 //
 // This grid is the programmatic dependent of what precedes it, typically the
-// previous decode call, and may start while that call is still running. Until
-// that call has completed (griddepcontrol.wait) nothing in global memory is
-// written. With `plan_staged` the list is built in shared memory before the
-// wait, from the context lengths (which nothing still running writes), and
-// only stored to the workspace after it; otherwise the plan waits first.
+// previous decode call, and may start while that call is still running. It
+// waits for that grid to complete (griddepcontrol.wait) before it reads or
+// writes global memory: the context lengths may come from the kernel before
+// it, and the workspace may still be in use by the previous call.
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
   constexpr int NW = PLAN_THREADS / 32;
-  extern __shared__ uint2 staged_list[];     // [list capacity] when a.plan_staged
   __shared__ int wsum[NW];
   __shared__ int hist[PLAN_BUCKETS];        // count, then running start of each size class
   __shared__ int wcnt[NW][PLAN_BUCKETS];    // per-warp counts of a round, then their offsets
@@ -177,9 +174,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   __shared__ int total_s;
   __shared__ int bad_len;  // a context length was clamped: reported after the wait
   pdl_launch_dependents();  // the decode grid may launch; it waits for this grid to finish
-  const bool staged = a.plan_staged != 0;
-  if (!staged) pdl_wait();
-  uint2 *const list = staged ? staged_list : a.work;
+  pdl_wait();
+  uint2 *const list = a.work;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs, P = a.part_tokens;
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
@@ -291,10 +287,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     if (bkt >= 0) list[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
     __syncthreads();  // wcnt and total_m_s are rewritten by the next round
   }
-  if (staged) pdl_wait();  // the previous call has completed: the workspace is free
   const int total = total_s;
-  if (staged)
-    for (int i = tid; i < total; i += PLAN_THREADS) a.work[i] = staged_list[i];
   if (a.merge_cnt) {
     const int n1 = S * a.num_kv_heads * a.max_chunks;
     for (int i = tid; i < n1; i += PLAN_THREADS) a.merge_cnt[i] = 0;
@@ -1108,21 +1101,10 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
-  // Lists that fit are built in the plan's shared memory before it waits for
-  // the previous call (see plan_kernel).
-  const long long list_cap = (long long)a.num_seqs * a.max_parts;
-  b.plan_staged = list_cap <= PLAN_STAGED_ENTRIES ? 1 : 0;
-  static bool plan_smem_set = false;
-  if (!plan_smem_set) {
-    e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PLAN_STAGED_ENTRIES * (int)sizeof(uint2));
-    if (e != cudaSuccess) return e;
-    plan_smem_set = true;
-  }
   cudaLaunchConfig_t pcfg = {};
   pcfg.gridDim = dim3(1);
   pcfg.blockDim = dim3(PLAN_THREADS);
-  pcfg.dynamicSmemBytes = b.plan_staged ? (size_t)list_cap * sizeof(uint2) : 0;
+  pcfg.dynamicSmemBytes = 0;
   pcfg.stream = stream;
   pcfg.attrs = attr;
   pcfg.numAttrs = 1;

@@ -46,7 +46,6 @@ struct DecodeArgs {
   int grid;            // CTAs of the decode grid (each takes item blockIdx.x first)
   int unit8;           // 1 when block_size % 16 == 8: a 16-token tile is two 8-token units
                        // that may sit in different blocks
-  int plan_staged;     // 1: the plan builds the list in shared memory before it waits
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level

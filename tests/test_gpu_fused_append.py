@@ -106,3 +106,40 @@ def test_output_into_pinned_host_memory(fused, part):
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     assert torch.equal(dev_out.cpu().view(torch.int16), host_out.view(torch.int16))
+
+
+@pytest.mark.parametrize("part", [0, 64])
+def test_lengths_advanced_on_device_just_before_each_call(part):
+    """A serving loop advances the context lengths with a device kernel on the
+    same stream right before each fused call. Every call must attend over the
+    new lengths and append at the new last slot."""
+    Hq, Hkv, D, B, S, steps = 8, 2, 128, 16, 24, 6
+    dt = torch.bfloat16
+    g = torch.Generator().manual_seed(11)
+    lens0 = torch.randint(1, 200, (S,), generator=g, dtype=torch.int32)
+    maxlen = int(lens0.max()) + steps
+    nb = -(-maxlen // B)
+    tables = torch.randperm(S * nb, generator=g).to(torch.int32).view(S, nb)
+    kc = torch.randn(S * nb, Hkv, B, D, generator=g).to(dt)
+    vc = torch.randn(S * nb, Hkv, B, D, generator=g).to(dt)
+    kd, vd, bt = kc.to(DEV), vc.to(DEV), tables.to(DEV)
+    lens = (lens0 - 1).to(DEV)  # the loop adds one before each call
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for step in range(steps):
+        q = torch.randn(S, Hq, D, generator=g).to(dt)
+        kn = torch.randn(S, Hkv, D, generator=g).to(dt)
+        vn = torch.randn(S, Hkv, D, generator=g).to(dt)
+        qd, knd, vnd = q.to(DEV), kn.to(DEV), vn.to(DEV)
+        out = torch.empty_like(qd)
+        lens.add_(1)  # the kernel just before the call writes the lengths
+        pkv.paged_attn_decode_append(out, qd, knd, vnd, kd, vd, bt, lens, D ** -0.5, maxlen,
+                                     partition_size=part, err=err)
+        L = (lens0 + step).to(torch.int64)
+        slots = tables[torch.arange(S), (L - 1) // B].to(torch.int64) * B + (L - 1) % B
+        oracle.cache_append(kc, vc, kn, vn, slots)
+        ref = oracle.paged_decode(q, kc, vc, tables, L.to(torch.int32), D ** -0.5)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0, f"step {step}"
+        assert_close_to_oracle(out, ref, dt, f"device-advanced lengths, step {step}")
+    assert torch.equal(kd.cpu().view(torch.int16), kc.view(torch.int16))
+    assert torch.equal(vd.cpu().view(torch.int16), vc.view(torch.int16))
