@@ -506,6 +506,10 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   if (warp == NCW) {
     // ======================= scheduler warp =======================
+    // The first item of every CTA is fixed. Its entry lies inside the list's
+    // capacity (grid <= capacity x Hkv), so it is loaded together with the
+    // list length instead of after it; it is used only if the item exists.
+    const uint2 first_wk = a.work[blockIdx.x / Hkv];
     const long long list_cap = (long long)a.num_seqs * a.max_parts;
     const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
     const int end_phase = total_items - END_ITEMS_PER_CTA * (int)gridDim.x;
@@ -516,7 +520,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                                  ? *reinterpret_cast<volatile const int32_t *>(a.err)
                                  : 0;
     bool first_post = true;
-    int item = blockIdx.x;  // the first item of every CTA is fixed; the counter starts at grid
+    int item = blockIdx.x;  // the counter starts at grid
     bool claimed = true;  // `item` holds an index taken from the work list
     int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
     uint32_t it = 0;      // descriptors posted
@@ -607,7 +611,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       // Items are entry-major: the KV heads of one entry are consecutive items.
       // A block's heads are contiguous in the pool, so CTAs working on
       // neighbouring items read neighbouring 4 KB slices (open DRAM rows).
-      const uint2 wk = a.work[item / Hkv];
+      const uint2 wk = first_post ? first_wk : a.work[item / Hkv];  // first_post: item == blockIdx.x
       const int h = item - (item / Hkv) * Hkv;
       const int s = min(static_cast<int>(wk.x >> 16), a.num_seqs - 1);
       const int p = static_cast<int>(wk.x & 0xffffu);
@@ -1025,13 +1029,13 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
         const float mw = comb[w * Shape::CW_FLOATS + NH * AS + n];
-        f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
+        f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
         den += f[w] * comb[w * Shape::CW_FLOATS + NH * AS + NH + n];
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) scales[n * NCW + w] = f[w] * inv;
-      scales[NH * NCW + n] = den > 0.f ? M + log2f(den) : -INFINITY;
+      scales[NH * NCW + n] = den > 0.f ? M + lg2_approx(den) : -INFINITY;
     }
     consumers_sync();
     // 3) outputs

@@ -206,6 +206,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// The hardware base-2 logarithm (PTX lg2.approx.ftz.f32).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <typename T>
 __device__ __forceinline__ T from_float(float x);
 template <>
