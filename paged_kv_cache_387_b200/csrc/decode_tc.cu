@@ -19,9 +19,9 @@
 //   also resets the dispatch and merge counters. The decode kernel is
 //   persistent, two CTAs per SM. Each CTA takes item blockIdx.x first, then
 //   pulls items (pair x KV head) from an atomic counter until the list is
-//   exhausted. Launches chain by programmatic dependence: the plan starts
-//   while the previous call finishes, and the decode grid's set-up overlaps
-//   the plan.
+//   exhausted. Launches chain by programmatic dependence: the plan is
+//   launched while the previous call finishes (and waits for it before it
+//   reads anything), and the decode grid's set-up overlaps the plan.
 //
 // Warp roles
 //   Warp 4 is the scheduler. It resolves items ahead of use and posts them as
@@ -64,9 +64,10 @@
 // partition, and otherwise to the workspace as (normalised o_p,
 // log2-sum-exp). The consumers meet at three barriers per item: a vote at
 // its start (which also orders the reuse of the combine area), one after
-// their partial rows are stored and one after the per-warp weights are. Every wait is bounded: one that gives up
-// sets an error status and a CTA-wide stop flag, and the kernel winds down,
-// first waiting (bounded) for the copies it still has in flight.
+// their partial rows are stored and one after the per-warp weights are.
+// Every wait is bounded: one that gives up sets an error status and a
+// CTA-wide stop flag, and the kernel winds down, first waiting (bounded) for
+// the copies it still has in flight.
 #include "pkv_device.cuh"
 #include "pkv_internal.h"
 
