@@ -84,6 +84,30 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_context_len, int partition_size);
 
 /*
+ * partition_size value that lets the library choose the partition length from
+ * the batch shape (see pkv_resolve_partition). Accepted by every decode call
+ * and by pkv_decode_workspace_bytes, which resolve it the same way.
+ */
+#define PKV_PARTITION_AUTO (-1)
+
+/*
+ * The partition length a decode call uses for partition_size.
+ *
+ * Splitting a context into partitions (page "PagedAttention Analysis",
+ * section 3: attention over any split of the tokens recombines exactly by
+ * log-sum-exp weights) is what lets a small batch of long contexts spread over
+ * all SMs. PKV_PARTITION_AUTO asks for about 1024 (sequence, partition, query
+ * head) rows in total, i.e. about one wave of work items at 4 query heads per
+ * KV head: with L = max(max_context_len, 1) and
+ * n = ceil(1024 / (num_seqs * num_heads)), it returns ceil(L / n) rounded up to
+ * a multiple of 16 and clamped to [256, 2048]. A batch of 32 or more sequences
+ * of 32 heads therefore gets 2048-token partitions, and one sequence of 4096
+ * tokens gets 256-token ones. Any other partition_size is returned unchanged.
+ * Pure arithmetic: it does not touch the GPU.
+ */
+int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int partition_size);
+
+/*
  * paged_attn_decode - one decode step of attention over a paged KV cache.
  *
  * For every sequence s and query head h, with G = num_heads / num_kv_heads,
@@ -117,7 +141,9 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
  *                grid and the workspace, so the call needs no device-to-host read.
  * scale          score multiplier; 1/sqrt(head_dim) gives the usual attention.
  * partition_size tokens per partition. 0 means no split (one partition of
- *                the whole context). Otherwise a positive multiple of 16.
+ *                the whole context), PKV_PARTITION_AUTO lets the library
+ *                choose (pkv_resolve_partition). Otherwise a positive
+ *                multiple of 16.
  * workspace      device scratch of at least pkv_decode_workspace_bytes(...)
  *                bytes, 256-byte aligned. Its contents on entry do not
  *                matter. Calls that overlap in time must not share it.

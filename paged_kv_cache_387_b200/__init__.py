@@ -27,11 +27,12 @@ DEV_ERRORS = {1: "block id out of range", 2: "append slot out of range",
               3: "copy or swap pair out of range", 4: "context length above max_context_len",
               5: "copy wait timed out"}
 DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
-DEFAULT_PARTITION = 2048  # tokens per split-context partition (measured best on B200)
+PARTITION_AUTO = -1  # the library picks the partition length from the batch shape
+DEFAULT_PARTITION = PARTITION_AUTO
 
 EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
            "kv_block_copy", "kv_block_swap", "pkv_check_wait_timeout",
-           "pkv_decode_workspace_bytes", "pkv_status_string")
+           "pkv_decode_workspace_bytes", "pkv_resolve_partition", "pkv_status_string")
 
 
 class PkvError(RuntimeError):
@@ -69,6 +70,8 @@ def load_library():
     lib.pkv_check_wait_timeout.restype = I
     lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.pkv_decode_workspace_bytes.restype = Z
+    lib.pkv_resolve_partition.argtypes = [I, I, I, I]
+    lib.pkv_resolve_partition.restype = I
     lib.pkv_status_string.argtypes = [I]
     lib.pkv_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -114,6 +117,13 @@ def decode_workspace_bytes(num_seqs: int, num_heads: int, head_dim: int, max_con
                            partition_size: int = DEFAULT_PARTITION) -> int:
     return int(load_library().pkv_decode_workspace_bytes(num_seqs, num_heads, head_dim,
                                                          max_context_len, partition_size))
+
+
+def resolve_partition(num_seqs: int, num_heads: int, max_context_len: int,
+                      partition_size: int = DEFAULT_PARTITION) -> int:
+    """The partition length a decode call uses (``PARTITION_AUTO`` resolved)."""
+    return int(load_library().pkv_resolve_partition(num_seqs, num_heads, max_context_len,
+                                                    partition_size))
 
 
 def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,

@@ -126,8 +126,21 @@ const char *pkv_status_string(int status) {
   }
 }
 
+int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int partition_size) {
+  if (partition_size != PKV_PARTITION_AUTO) return partition_size;
+  constexpr long long kRows = 1024, kMin = 256, kMax = 2048;
+  const long long rows = (long long)(num_seqs > 0 ? num_seqs : 1) * (num_heads > 0 ? num_heads : 1);
+  const long long n = (kRows + rows - 1) / rows;  // partitions wanted per sequence
+  const long long L = max_context_len > 0 ? max_context_len : 1;
+  long long part = ((L + n - 1) / n + 15) / 16 * 16;
+  if (part < kMin) part = kMin;
+  if (part > kMax) part = kMax;
+  return (int)part;
+}
+
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
                                   int partition_size) {
+  partition_size = pkv_resolve_partition(num_seqs, num_heads, max_context_len, partition_size);
   if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
       partition_size < 0)
     return 0;
@@ -147,6 +160,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
                 int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
                 int dtype, int partition_size, void *workspace, size_t workspace_bytes,
                 int32_t *err, void *stream, const void *k_new, const void *v_new) {
+  partition_size = pkv_resolve_partition(num_seqs, num_heads, max_context_len, partition_size);
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
       partition_size < 0)

@@ -68,6 +68,30 @@ def test_workspace_arithmetic(lib):
     assert f(0, 32, 128, 512, 512) == 0
 
 
+def test_auto_partition_rule(lib):
+    r = lib.pkv_resolve_partition
+    AUTO = pkv.PARTITION_AUTO
+    # explicit sizes pass through
+    assert r(1, 32, 4096, 512) == 512 and r(1, 32, 4096, 0) == 0
+    # big batches: 2048-token partitions (one partition when the contexts are shorter)
+    assert r(256, 32, 4096, AUTO) == 2048
+    assert r(64, 40, 2048, AUTO) == 2048
+    assert r(256, 32, 100, AUTO) == 256
+    # small batches: about 1024 (sequence, partition, head) rows, partitions >= 256 tokens
+    assert r(1, 32, 4096, AUTO) == 256       # n = 32 -> 128 tokens -> raised to 256
+    assert r(1, 32, 32768, AUTO) == 1024     # n = 32 -> 1024
+    assert r(1, 32, 131072, AUTO) == 2048    # n = 32 -> 4096 -> lowered to 2048
+    assert r(2, 32, 20000, AUTO) == 1264     # n = 16 -> 1250 -> multiple of 16
+    assert r(4, 32, 16384, AUTO) == 2048     # n = 8 -> 2048
+    assert r(8, 8, 3000, AUTO) == 256        # n = 16 -> 188 -> 256
+    assert r(0, 32, 0, AUTO) == 256          # degenerate shapes stay valid
+    for S, Hq, L in [(1, 32, 4096), (3, 8, 70000), (256, 32, 4096), (5, 40, 2000)]:
+        assert r(S, Hq, L, AUTO) % 16 == 0
+        assert (lib.pkv_decode_workspace_bytes(S, Hq, 128, L, AUTO)
+                == lib.pkv_decode_workspace_bytes(S, Hq, 128, L, r(S, Hq, L, AUTO)))
+    assert pkv.resolve_partition(1, 32, 4096) == 256  # the binding's default is AUTO
+
+
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below is rejected first
 
 
@@ -83,6 +107,8 @@ def test_decode_argument_checks(lib):
     assert decode(lib, out=None) == pkv.PKV_EINVAL
     assert decode(lib, Hq=6, Hkv=4) == pkv.PKV_EINVAL
     assert decode(lib, part=24) == pkv.PKV_EINVAL
+    assert decode(lib, part=-2) == pkv.PKV_EINVAL                     # only -1 means AUTO
+    assert decode(lib, part=pkv.PARTITION_AUTO, L=200000, ws=None, wsb=0) == pkv.PKV_EINVAL
     assert decode(lib, dtype=7) == pkv.PKV_EINVAL
     assert decode(lib, scale=float("nan")) == pkv.PKV_EINVAL
     assert decode(lib, L=2048, ws=None, wsb=0) == pkv.PKV_EINVAL     # workspace needed

@@ -47,6 +47,12 @@ def test_fused_append_decode_matches_append_then_decode(dt, D, B, Hq, Hkv, part)
     fused_vs_oracle(c, part, f"{dt} D{D} B{B} G{Hq // Hkv} p{part}")
 
 
+def test_fused_append_auto_partition():
+    c = make_random_case("fused_auto", 32, 8, 128, 16, [4096, 50, 1], torch.bfloat16, seed=9,
+                         device=DEV, with_append=True)
+    fused_vs_oracle(c, pkv.PARTITION_AUTO, "fused, auto partition")
+
+
 def test_fused_append_opt13b_workload():
     c = make_case("opt13b_mha_b64", device=DEV)
     fused_vs_oracle(c, c.partition_size, "opt13b fused")

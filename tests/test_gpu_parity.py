@@ -59,6 +59,21 @@ def test_block_size_64_and_256():
         assert_close_to_oracle(gpu_decode(c), oracle_decode(c), torch.bfloat16, f"B{B}")
 
 
+@pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("lens", [[4096], [3000, 1, 7001], [20000, 5, 900, 16, 333]])
+def test_auto_partition_small_batches(dt, lens):
+    """PARTITION_AUTO splits a small batch of long contexts into short
+    partitions (256 tokens for one 4096-token sequence of 8 heads; 26
+    partitions, two merge levels, for the 20000-token one); the result must
+    still match the oracle."""
+    D = 64 if dt == "f32" else 128
+    c = make_random_case("auto", 8, 2, D, 16, lens, DT[dt], seed=len(lens) + D, device=DEV)
+    part = pkv.resolve_partition(c.num_seqs, c.num_heads, c.max_context_len)
+    assert 256 <= part < max(lens)  # the contexts are split
+    got = gpu_decode(c, partition_size=pkv.PARTITION_AUTO)
+    assert_close_to_oracle(got, oracle_decode(c), DT[dt], f"{dt} auto partition {part}")
+
+
 def test_placement_invariance_and_contiguous_equality():
     kw = dict(name="perm", num_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
               context_lens=[3, 77, 300, 1030], dtype=torch.bfloat16, seed=55, device=DEV,
