@@ -43,7 +43,7 @@
 //     - block sizes that are odd multiples of 8: two 8-row boxes per
 //       64-element half, one per 8-token unit, each from its own block.
 //   The boxes are 128-byte swizzled. The fill runs ahead of the warp's math
-//   across item boundaries. No load uses cluster multicast.
+//   across item boundaries. Every load lands in the issuing CTA only.
 //
 // Math (per tile, per consumer warp), fp32 accumulation:
 //   S^T[16 tok][8] = K_tile[16][D] . Q^T[D][8]  mma.sync m16n8k16. K is the A

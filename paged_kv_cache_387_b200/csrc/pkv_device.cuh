@@ -77,7 +77,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 // Wait until the grids this one depends on have completed.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// ---- TMA (tiled, no multicast) --------------------------------------------
+// ---- TMA (tiled, single-CTA destination) ----------------------------------
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint32_t bar) {
   asm volatile(
