@@ -618,9 +618,14 @@ def run_ours(args, rank, world, local_rank):
     host_outs = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(nb)]
     d2h = host_outs[0].numel() * host_outs[0].element_size()
     h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    # Per buffer b: in_ready (upload done), done (decode done), out_free
+    # (download done, which follows `done`). The upload into buffer b waits
+    # for out_free of the step that used b before, so the compute stream
+    # only waits for in_ready and records done: one stream operation on each
+    # side of a decode call, which keeps most of the programmatic launch
+    # overlap between consecutive calls.
     in_ready = [torch.cuda.Event() for _ in range(nb)]
-    in_free = [torch.cuda.Event() for _ in range(nb)]
-    out_ready = [torch.cuda.Event() for _ in range(nb)]
+    done = [torch.cuda.Event() for _ in range(nb)]
     out_free = [torch.cuda.Event() for _ in range(nb)]
 
     def run_step(inp, o):
@@ -641,25 +646,22 @@ def run_ours(args, rank, world, local_rank):
             b = i % nb
             with torch.cuda.stream(h2d_stream):
                 if i >= nb:
-                    h2d_stream.wait_event(in_free[b])
+                    h2d_stream.wait_event(out_free[b])  # buffer b's previous step is over
                 elif start_event is not None:
                     h2d_stream.wait_event(start_event)
                 dev_stage[b].copy_(host_stage, non_blocking=True)
                 in_ready[b].record(h2d_stream)
             stream.wait_event(in_ready[b])
-            if i >= nb:
-                stream.wait_event(out_free[b])
             if args.e2e_result_in_host_memory:
                 # the decode writes its result straight into pinned host memory
                 run_step(dev_sets[b], host_outs[b])
-                in_free[b].record(stream)
-                out_free[b].record(stream)
+                done[b].record(stream)
+                out_free[b] = done[b]
                 continue
             run_step(dev_sets[b], outs[b])
-            in_free[b].record(stream)
-            out_ready[b].record(stream)
+            done[b].record(stream)
             with torch.cuda.stream(d2h_stream):
-                d2h_stream.wait_event(out_ready[b])
+                d2h_stream.wait_event(done[b])
                 host_outs[b].copy_(outs[b], non_blocking=True)
                 out_free[b].record(d2h_stream)
         last = torch.cuda.Event()
