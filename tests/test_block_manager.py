@@ -8,7 +8,6 @@ import numpy as np
 import pytest
 
 from pkv_inputs import BlockAllocator, kv_bytes_per_token, make_shared_prefix_case
-from pkv_inputs.block_manager import SeqState
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
 

@@ -2,7 +2,6 @@
 the pool after the call must equal the oracle's append bit for bit, and the
 output must match the oracle's decode over the appended cache."""
 
-import numpy as np
 import pytest
 import torch
 

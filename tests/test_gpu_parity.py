@@ -1,6 +1,5 @@
 """Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle."""
 
-import math
 
 import numpy as np
 import pytest

@@ -3,7 +3,6 @@ oracle: the swap space after a swap-out, and the device pool after a swap-in,
 must equal the oracle's block swap bit for bit, and a decode after the round
 trip (into other physical blocks) must give the same output as before."""
 
-import numpy as np
 import pytest
 import torch
 
