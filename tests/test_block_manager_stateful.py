@@ -13,6 +13,12 @@ swap-out / swap-in steps over a tiny pool and, after every step, checks:
 * tables: ceil(num_tokens / B) entries per sequence;
 * contents: the block copies and moves the allocator returns, applied to a
   simulated pool of token ids, keep every sequence's logical tokens intact.
+
+A second machine does the same for the prefix cache (page "PagedAttention
+Analysis", section 4: blocks keyed by a hash of the whole prefix, shared
+through a global table): requests over a two-letter alphabet collide often,
+and every cache hit must serve a block that holds exactly the requested
+tokens, also after cached blocks were released, evicted and reused.
 """
 
 from collections import Counter
@@ -21,7 +27,7 @@ from hypothesis import settings
 from hypothesis import strategies as st
 from hypothesis.stateful import RuleBasedStateMachine, invariant, precondition, rule
 
-from pkv_inputs import BlockAllocator, SwapSpace
+from pkv_inputs import BlockAllocator, PrefixCache, SwapSpace
 
 P, B = 24, 4
 
@@ -152,3 +158,56 @@ class BlockBookkeeping(RuleBasedStateMachine):
 
 TestBlockBookkeeping = BlockBookkeeping.TestCase
 TestBlockBookkeeping.settings = settings(max_examples=150, stateful_step_count=40, deadline=None)
+
+
+class PrefixCacheBookkeeping(RuleBasedStateMachine):
+    def __init__(self):
+        super().__init__()
+        self.alloc = BlockAllocator(16, B, free_order=list(range(16))[::-1])
+        self.cache = PrefixCache(self.alloc)
+        self.data = {}   # block -> the B tokens written into it
+        self.seqs = []
+        self.tokens = []
+
+    @rule(toks=st.lists(st.integers(0, 1), min_size=1, max_size=14))
+    def request(self, toks):
+        nb = -(-len(toks) // B)
+        if self.alloc.num_free < nb:
+            return
+        hits0 = self.cache.hits
+        seq, fills = self.cache.new_sequence(toks)
+        assert len(seq.table) == nb
+        full = len(toks) // B
+        for j, b in enumerate(seq.table):
+            want = toks[j * B:(j + 1) * B]
+            if j in fills:
+                self.data[b] = list(want)          # the caller fills misses and the tail
+            else:
+                assert j < full                     # only full blocks are shared
+                assert self.data.get(b) == want     # a hit holds exactly these tokens
+        assert self.cache.hits - hits0 == nb - len(fills)
+        self.seqs.append(seq)
+        self.tokens.append(list(toks))
+
+    @precondition(lambda self: self.seqs)
+    @rule(pick=st.integers(0, 10 ** 6))
+    def release(self, pick):
+        i = pick % len(self.seqs)
+        self.cache.release(self.seqs[i])
+        del self.seqs[i], self.tokens[i]
+
+    @invariant()
+    def refcounts_keys_and_contents(self):
+        refs = Counter(b for s in self.seqs for b in s.table)
+        for b in range(self.alloc.num_blocks):
+            assert self.alloc.refcount(b) == refs.get(b, 0), b
+        assert self.alloc.num_free == self.alloc.num_blocks - len(refs)
+        assert {b: k for k, b in self.cache.table.items()} == self.cache.key_of
+        for seq, toks in zip(self.seqs, self.tokens):
+            got = [self.data[seq.table[t // B]][t % B] for t in range(len(toks))]
+            assert got == toks
+
+
+TestPrefixCacheBookkeeping = PrefixCacheBookkeeping.TestCase
+TestPrefixCacheBookkeeping.settings = settings(max_examples=150, stateful_step_count=40,
+                                               deadline=None)
