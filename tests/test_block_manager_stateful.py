@@ -19,15 +19,21 @@ Analysis", section 4: blocks keyed by a hash of the whole prefix, shared
 through a global table): requests over a two-letter alphabet collide often,
 and every cache hit must serve a block that holds exactly the requested
 tokens, also after cached blocks were released, evicted and reused.
+
+Beam search (section 4 of the same page: the beams share the prompt and
+intermediate blocks, and the sharing changes every step) is checked the same
+way: with random parents every step, each beam must read back its parent's
+tokens plus its own new one once the step's copies have run before its
+writes, and releasing the request must free every block.
 """
 
 from collections import Counter
 
-from hypothesis import settings
+from hypothesis import given, settings
 from hypothesis import strategies as st
 from hypothesis.stateful import RuleBasedStateMachine, invariant, precondition, rule
 
-from pkv_inputs import BlockAllocator, PrefixCache, SwapSpace
+from pkv_inputs import BeamSearch, BlockAllocator, PrefixCache, SwapSpace
 
 P, B = 24, 4
 
@@ -211,3 +217,33 @@ class PrefixCacheBookkeeping(RuleBasedStateMachine):
 TestPrefixCacheBookkeeping = PrefixCacheBookkeeping.TestCase
 TestPrefixCacheBookkeeping.settings = settings(max_examples=150, stateful_step_count=40,
                                                deadline=None)
+
+
+@settings(max_examples=200, deadline=None)
+@given(width=st.integers(1, 4), prompt=st.integers(1, 10),
+       parents=st.lists(st.lists(st.integers(0, 3), min_size=4, max_size=4), max_size=12))
+def test_beam_search_contents_and_no_leaks(width, prompt, parents):
+    P_beam = width * (-(-(prompt + len(parents)) // B) + 1)
+    alloc = BlockAllocator(P_beam, B, free_order=list(range(P_beam))[::-1])
+    bs = BeamSearch(alloc, prompt, width)
+    data = {}
+    root = bs.beams[0]
+    toks = [list(range(prompt)) for _ in range(width)]
+    for t in range(prompt):
+        data.setdefault(root.table[t // B], [None] * B)[t % B] = t
+    nxt = prompt
+    for step, ps in enumerate(parents):
+        ps = [p % width for p in ps[:width]]
+        slots, copies = bs.step(ps)
+        for cp in copies:  # every copy runs before any of the step's writes
+            data[cp.dst] = list(data[cp.src])
+        toks = [toks[p] + [nxt + i] for i, p in enumerate(ps)]
+        for i, slot in enumerate(slots):
+            data.setdefault(slot // B, [None] * B)[slot % B] = nxt + i
+        nxt += width
+        for beam, want in zip(bs.beams, toks):
+            assert beam.num_tokens == len(want)
+            got = [data[beam.table[t // B]][t % B] for t in range(beam.num_tokens)]
+            assert got == want, f"step {step}"
+    bs.release()
+    assert alloc.num_free == P_beam
