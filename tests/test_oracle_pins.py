@@ -24,6 +24,9 @@ import pytest
 import torch
 import torch.nn.functional as F
 
+from hypothesis import given, settings
+from hypothesis import strategies as st
+
 import oracle
 
 DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
@@ -277,3 +280,27 @@ def test_block_swap_is_numpy_block_assignment():
         assert torch.equal(dst_v.view(bits), ev.view(bits))
         with pytest.raises(RuntimeError):
             oracle.block_swap(dst_k, dst_v, src_k, src_v, np.array([[9, 0]], dtype=np.int32))
+
+
+@settings(max_examples=60, deadline=None)
+@given(lens=st.lists(st.integers(1, 70), min_size=1, max_size=4),
+       B=st.sampled_from([1, 3, 8, 16]), Hkv=st.integers(1, 2), G=st.integers(1, 3),
+       D=st.sampled_from([8, 16, 64]), dt=st.sampled_from(["f32", "f16", "bf16"]),
+       scale=st.floats(0.0, 1.0), seed=st.integers(0, 2 ** 16), part=st.sampled_from([1, 5, 32]))
+def test_random_shapes_equal_contiguous_library_attention(lens, B, Hkv, G, D, dt, scale, seed,
+                                                           part):
+    """The library-routine pin over random shapes, block sizes, group sizes,
+    dtypes, scales and placements; the partitioned form (partitions of `part`
+    blocks) agrees too."""
+    dtype = DT[dt]
+    ks, vs = dense_tokens(lens, Hkv, D, dtype, seed=seed)
+    q = torch.randn(len(lens), Hkv * G, D,
+                    generator=torch.Generator().manual_seed(seed + 1)).to(dtype)
+    nb = sum(-(-L // B) for L in lens) + 3
+    perm = np.random.default_rng(seed).permutation(nb)
+    k_pool, v_pool, bt, cl = page_tokens(ks, vs, B, nb, perm)
+    got = oracle.paged_decode(q, k_pool, v_pool, bt, cl, scale)
+    ref = sdpa_reference(q, ks, vs, scale)
+    assert np.abs(got - ref).max() < 1e-12
+    split, _, _ = oracle.paged_decode_partitioned(q, k_pool, v_pool, bt, cl, scale, part * B)
+    assert np.abs(split - got).max() < 1e-12
