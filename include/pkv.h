@@ -1,7 +1,7 @@
 /*
  * pkv.h - C ABI of the paged KV-cache decode library (sm_100a).
  *
- * Three operations on a KV cache split into fixed-size blocks that sit
+ * Operations on a KV cache split into fixed-size blocks that sit
  * non-contiguously in one physical pool per K and V:
  *
  *   paged_attn_decode  single-query attention of every sequence over its
@@ -14,11 +14,12 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * Pointers. Every data pointer is a DEVICE pointer owned by the caller, with
- * one exception: the `out` of the decode entry points may also be page-locked
- * host memory that the device addresses directly (unified addressing, e.g.
- * from cudaHostAlloc). The kernels then write the result over the bus with
- * plain stores, and no separate device-to-host copy is needed; the caller
- * reads it once the stream has passed the call. The library never allocates,
+ * two exceptions. The `out` of the decode entry points, and the four pools of
+ * kv_block_swap, may also be page-locked host memory that the device
+ * addresses directly (unified addressing, e.g. from cudaHostAlloc). The
+ * kernels then move the data over the bus with plain loads and stores, and
+ * no separate copy is needed; the caller reads a result once the stream has
+ * passed the call. The library never allocates,
  * frees or retains memory. Block allocation is host
  * bookkeeping over integer block ids, and needs no device allocation during
  * generation (page "추론 엔진에서의 메모리 가상화", molayo1419.me, block
