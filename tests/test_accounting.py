@@ -3,7 +3,7 @@
 The decode's algorithmic bytes per sequence of L tokens are the K and V of
 its valid tokens once per KV head (2*L*Hkv*D*sz), q in and o out
 (2*Hq*D*sz), and its table entries and length (4*ceil(L/B) + 4); empty
-reserved slots are not counted (page "PagedAttention Analysis", section 1:
+reserved slots are not counted (page "PagedAttention Analysis", section 2:
 the waste paging avoids is at most the unfilled part of a last block).
 """
 
