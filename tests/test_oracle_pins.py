@@ -259,6 +259,49 @@ def test_block_copy_matches_numpy_slices():
     assert np.array_equal(v_pool.view(torch.int16).numpy(), ev)
 
 
+def test_append_out_of_range_slot_is_skipped_and_reported():
+    """A slot at or past num_blocks * B names no pool slot: the oracle skips that
+    token, still writes every other token (the numpy scatter of the valid ones)
+    and reports the error."""
+    rng = np.random.default_rng(6)
+    P, Hkv, B, D, T = 6, 2, 8, 16, 5
+    k_pool = torch.from_numpy(rng.standard_normal((P, Hkv, B, D)).astype(np.float32)).bfloat16()
+    v_pool = torch.from_numpy(rng.standard_normal((P, Hkv, B, D)).astype(np.float32)).bfloat16()
+    k_new = torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).bfloat16()
+    v_new = torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).bfloat16()
+    slots = np.array([3, P * B, 17, P * B + 40, P * B - 1], dtype=np.int64)
+    ek = k_pool.view(torch.int16).numpy().copy()
+    ev = v_pool.view(torch.int16).numpy().copy()
+    for i, sl in enumerate(slots):
+        if sl < P * B:
+            ek[sl // B, :, sl % B, :] = k_new.view(torch.int16).numpy()[i]
+            ev[sl // B, :, sl % B, :] = v_new.view(torch.int16).numpy()[i]
+    with pytest.raises(RuntimeError, match="out of range"):
+        oracle.cache_append(k_pool, v_pool, k_new, v_new, torch.from_numpy(slots))
+    assert np.array_equal(k_pool.view(torch.int16).numpy(), ek)
+    assert np.array_equal(v_pool.view(torch.int16).numpy(), ev)
+
+
+@pytest.mark.parametrize("bad", [[12, 3], [-1, 3], [2, 12], [2, -5]])
+def test_block_copy_out_of_range_pair_is_skipped_and_reported(bad):
+    """A pair whose source or destination lies outside [0, num_blocks) is
+    skipped and reported; the in-range pairs around it are still copied."""
+    rng = np.random.default_rng(9)
+    P, Hkv, B, D = 12, 2, 16, 32
+    k_pool = torch.from_numpy(rng.standard_normal((P, Hkv, B, D)).astype(np.float32)).half()
+    v_pool = torch.from_numpy(rng.standard_normal((P, Hkv, B, D)).astype(np.float32)).half()
+    pairs = np.array([[1, 7], bad, [4, 9]], dtype=np.int32)
+    ek = k_pool.view(torch.int16).numpy().copy()
+    ev = v_pool.view(torch.int16).numpy().copy()
+    for s_, d_ in ([1, 7], [4, 9]):
+        ek[d_] = ek[s_]
+        ev[d_] = ev[s_]
+    with pytest.raises(RuntimeError, match="out of range"):
+        oracle.block_copy(k_pool, v_pool, torch.from_numpy(pairs))
+    assert np.array_equal(k_pool.view(torch.int16).numpy(), ek)
+    assert np.array_equal(v_pool.view(torch.int16).numpy(), ev)
+
+
 def test_block_swap_is_numpy_block_assignment():
     """oracle.block_swap copies whole blocks between two pools: the same as
     torch's indexed assignment dst[d] = src[s] per pair, bit for bit."""
