@@ -134,6 +134,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
                       err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """One decode step of paged attention; writes ``out`` [S][Hq][D]."""
     lib = load_library()
+    _dev_ptr(q, "q")  # q decides the device every other tensor must be on
     dev = q.device
     if q.dtype not in DTYPE_CODES or out.dtype != q.dtype or k_pool.dtype != q.dtype \
             or v_pool.dtype != q.dtype:
@@ -172,6 +173,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
     (``k_new[s]``, ``v_new[s]``, [S][Hkv][D]) is written into the pool slot of its
     token ``context_lens[s] - 1`` and attended over, in one pass (fp16/bf16)."""
     lib = load_library()
+    _dev_ptr(q, "q")  # q decides the device every other tensor must be on
     dev = q.device
     if q.dtype not in DTYPE_CODES or any(t.dtype != q.dtype
                                          for t in (out, k_new, v_new, k_pool, v_pool)):
