@@ -62,9 +62,16 @@ def parse_args():
                     help="also time the same batch with identity block placement")
     ap.add_argument("--e2e-buffers", type=int, default=3,
                     help="device input/output buffers in the end-to-end loop (>= 2)")
+    ap.add_argument("--e2e-compute-streams", type=int, default=1,
+                    help="compute streams that take turns with the end-to-end loop's steps, "
+                         "each with its own workspace (>= 1)")
     ap.add_argument("--e2e-result-in-host-memory", action="store_true",
                     help="end-to-end loop: the decode writes its result straight into pinned "
                          "host memory instead of a device buffer plus a device-to-host copy")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads' device-timed lines (OPT-13B, long split, "
+                         "shared prefix, beam search, prefix cache, identity placement, "
+                         "standalone append and copy)")
     ap.add_argument("--separate-append", action="store_true",
                     help="run kv_cache_append and paged_attn_decode as two calls instead of "
                          "the fused paged_attn_decode_append")
@@ -258,6 +265,14 @@ def step_bytes(case, nseq=None):
     return b, app
 
 
+def case_unique_kv_bytes(case):
+    """K/V bytes of the distinct physical blocks the step reads."""
+    from pkv_inputs import unique_kv_bytes
+    return unique_kv_bytes(case.block_tables.cpu().tolist(), case.context_lens.cpu().tolist(),
+                           case.block_size, case.num_kv_heads, case.head_dim,
+                           case.k_pool.element_size())
+
+
 def measure_swap(case, dev, stream, pkv, nseq=32, reps=5):
     """Swap the blocks of the batch's first `nseq` sequences out to a swap
     space in pinned host memory and back in (kv_block_swap, both directions),
@@ -338,7 +353,8 @@ def run_reference(args, rank, world):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(case, args.workload, args.gpus),
+        "config": dict(config_block(case, args.workload, args.gpus),
+                       call=call_description(case, args)),
         "seq_steps_per_s": nseq / dt,
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
@@ -346,6 +362,13 @@ def run_reference(args, rank, world):
                 "d2h_bytes_per_step": 0},
     }
     return line
+
+
+def call_description(case, args):
+    """The library call a step makes (the same text in both arms' config)."""
+    fused = not args.separate_append and case.q.dtype != __import__("torch").float32
+    return ("paged_attn_decode_append (append fused into the decode)" if fused else
+            "kv_cache_append + paged_attn_decode")
 
 
 def config_block(case, workload, n_gpus):
@@ -381,12 +404,13 @@ def config_block(case, workload, n_gpus):
 # our arm
 # ---------------------------------------------------------------------------
 
-def build_bench_case(args, dev, rank):
+def build_bench_case(args, dev, rank, workload=None):
     """The step's inputs, plus extra report fields for special workloads."""
     import torch
     from pkv_inputs import make_case
     from pkv_inputs.workloads import WORKLOADS, DecodeCase, make_shared_prefix_case
-    if args.workload == "beam_search":
+    workload = args.workload if workload is None else workload
+    if workload == "beam_search":
         # 32 requests x 4 beams, Llama-8B-shaped heads: after 127 steps with seeded
         # random parents, the timed step is the 128th (copies applied, then the
         # fused append + decode of all 128 beams).
@@ -394,18 +418,17 @@ def build_bench_case(args, dev, rank):
         case = make_beam_search_case(device=dev, seed=rank_seed(393, rank))
         m = case.meta
         per_tok = 2 * case.num_kv_heads * case.head_dim * case.k_pool.element_size()
-        per_blk = per_tok * case.block_size
         extras = {"beam_search": {
             "requests": m["requests"], "width": m["width"],
             "blocks_in_use": m["blocks_in_use"], "blocks_unshared": m["blocks_unshared"],
             "memory_saving": 1.0 - m["blocks_in_use"] / m["blocks_unshared"],
             "logical_kv_bytes": int(case.context_lens.sum()) * per_tok,
-            "unique_kv_bytes": m["blocks_in_use"] * per_blk,
-            "note": "value/roofline count logical bytes; blocks shared by the beams of a "
-                    "request are read from L2"}}
+            "unique_kv_bytes": case_unique_kv_bytes(case),
+            "note": "value/roofline count logical bytes; unique_kv_bytes counts each "
+                    "physical block the beams share once"}}
         case.meta = {k: v for k, v in m.items() if k not in ("allocator", "searches")}
         return case, extras
-    if args.workload == "prefix_cache":
+    if workload == "prefix_cache":
         # 64 requests: a 1024-token system prompt shared by all, 8 groups sharing a
         # 512-token prefix, unique 128-256-token suffixes; blocks from the prefix
         # cache; the timed step appends each request's last token and decodes.
@@ -418,14 +441,15 @@ def build_bench_case(args, dev, rank):
             "blocks_in_use": m["blocks_in_use"], "blocks_unshared": m["blocks_unshared"],
             "memory_saving": 1.0 - m["blocks_in_use"] / m["blocks_unshared"],
             "logical_kv_bytes": int(case.context_lens.sum()) * per_tok,
-            "unique_kv_bytes": m["blocks_in_use"] * per_tok * case.block_size,
-            "note": "value/roofline count logical bytes; cached prefix blocks are read "
-                    "from L2 by the requests that share them"}}
+            "unique_kv_bytes": case_unique_kv_bytes(case),
+            "note": "value/roofline count logical bytes; unique_kv_bytes counts each "
+                    "cached block the requests share once"}}
         case.meta = {k: v for k, v in m.items() if k not in ("cache", "tokens")}
         return case, extras
-    if args.workload != "shared_prefix":
-        case = make_case(args.workload, device=dev, with_append=True, num_seqs=args.num_seqs,
-                         seed=rank_seed(WORKLOADS[args.workload]["seed"], rank))
+    if workload != "shared_prefix":
+        case = make_case(workload, device=dev, with_append=True,
+                         num_seqs=args.num_seqs if workload == args.workload else None,
+                         seed=rank_seed(WORKLOADS[workload]["seed"], rank))
         return case, {}
     # 16 prompts x 6 samples sharing refcounted prompt blocks: the copy-on-write
     # block copies run once, then the samples decode 64 divergent tokens. The
@@ -459,26 +483,91 @@ def build_bench_case(args, dev, rank):
                       slot_mapping=st["slot_mapping"])
     # unique K/V bytes: the shared full prompt blocks once per prompt, plus every
     # sample's own blocks
-    bt = st["block_tables"].cpu()
     lens = st["context_lens"].cpu()
     per_tok = 2 * sp.num_kv_heads * sp.head_dim * sp.k_pool.element_size()
-    seen, unique_tokens = set(), 0
-    for s_ in range(bt.shape[0]):
-        L = int(lens[s_])
-        for j in range(-(-L // sp.block_size)):
-            phys = int(bt[s_, j])
-            if phys not in seen:
-                seen.add(phys)
-                unique_tokens += min(sp.block_size, L - j * sp.block_size)
     extras = {"block_copy": {"pairs": int(pairs.shape[0]), "ms": copy_ms,
+                             "us": copy_ms * 1e3,
                              "GB/s": copy_bytes / (copy_ms * 1e-3) / 1e9,
                              "bytes": copy_bytes},
               "shared_prefix": {"logical_kv_bytes": int(lens.sum()) * per_tok,
-                                "unique_kv_bytes": unique_tokens * per_tok,
+                                "unique_kv_bytes": case_unique_kv_bytes(case),
                                 "prompts": sp.num_prompts, "samples": sp.samples,
-                                "note": "value/roofline count logical bytes; blocks shared "
-                                        "by the samples of a prompt are read from L2"}}
+                                "note": "value/roofline count logical bytes; unique_kv_bytes "
+                                        "counts each block the samples of a prompt share "
+                                        "once"}}
     return case, extras
+
+EXTRA_WORKLOADS = ("opt13b_mha_b64", "long_split_b8", "shared_prefix", "beam_search",
+                   "prefix_cache")
+
+
+def time_fused_call(pkv, case, steps, warmup, stream):
+    """Device milliseconds of one paged_attn_decode_append call on `case`, the
+    mean over `steps` back-to-back calls after `warmup` (appending the same
+    newest token again leaves the pools unchanged)."""
+    import torch
+    dev = case.q.device
+    mcl = case.max_context_len
+    out = torch.empty_like(case.q)
+    wsb = pkv.decode_workspace_bytes(case.num_seqs, case.num_heads, case.head_dim, mcl,
+                                     case.partition_size)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        pkv.paged_attn_decode_append(out, case.q, case.k_new, case.v_new, case.k_pool,
+                                     case.v_pool, case.block_tables, case.context_lens,
+                                     case.scale, mcl, partition_size=case.partition_size,
+                                     workspace=ws, err=err)
+    for _ in range(max(3, warmup)):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word set: {pkv.device_error_message(int(err.item()))}")
+    return a.elapsed_time(b) / steps
+
+
+def extra_lines(args, dev, rank, pkv, stream, peak):
+    """The other workloads of the scope, each timed on the device like the
+    headline (the fused append + decode call, `--steps` calls after
+    `--warmup`): logical GB/s and, for the workloads that share blocks, the
+    GB/s of the distinct blocks read, with their fractions of the copy peak."""
+    import torch
+    lines = {}
+    for w in EXTRA_WORKLOADS:
+        if w == args.workload:
+            continue
+        case, ex = build_bench_case(args, dev, rank, workload=w)
+        ms = time_fused_call(pkv, case, args.steps, args.warmup, stream)
+        dec, app = step_bytes(case)
+        d = {"ms_per_step": ms, "GB/s": (dec + app) / (ms * 1e-3) / 1e9,
+             "frac": (dec + app) / (ms * 1e-3) / 1e9 / peak,
+             "seq_steps_per_s": case.num_seqs / (ms * 1e-3),
+             "num_seqs": case.num_seqs, "context_tokens": int(case.context_lens.sum()),
+             "partition_size": case.partition_size, "dtype": str(case.q.dtype)}
+        for key in ("shared_prefix", "beam_search", "prefix_cache"):
+            if key in ex:
+                info = ex[key]
+                # the unique step: each distinct block's K/V once, plus the q/o,
+                # table and append bytes of every sequence
+                ub = info["unique_kv_bytes"] + (dec + app - info["logical_kv_bytes"])
+                d.update({k: v for k, v in info.items() if k != "note"})
+                d["unique_bytes"] = ub
+                d["unique_GB/s"] = ub / (ms * 1e-3) / 1e9
+                d["unique_frac"] = d["unique_GB/s"] / peak
+        if "block_copy" in ex:
+            lines["block_copy"] = ex["block_copy"]
+        lines[w] = d
+        del case
+        torch.cuda.empty_cache()
+    return lines
+
 
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -619,26 +708,32 @@ def run_ours(args, rank, world, local_rank):
     h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     # Per buffer b: in_ready (upload done), done (decode done), out_free
     # (download done, which follows `done`). The upload into buffer b waits
-    # for out_free of the step that used b before, so the compute stream
-    # only waits for in_ready and records done: one stream operation on each
-    # side of a decode call, which keeps most of the programmatic launch
-    # overlap between consecutive calls.
+    # for out_free of the step that used b before, so a compute stream only
+    # waits for in_ready and records done. The steps take turns on
+    # `--e2e-compute-streams` compute streams, each with its own workspace:
+    # a stream operation between two calls on one stream ends the
+    # programmatic overlap of their launches, and with two streams the next
+    # step's kernels still start while the previous step's drain.
+    ncs = max(1, args.e2e_compute_streams)
+    comp = [stream] + [torch.cuda.Stream(dev) for _ in range(ncs - 1)]
+    wss = [ws] + [torch.empty_like(ws) for _ in range(ncs - 1)]
     in_ready = [torch.cuda.Event() for _ in range(nb)]
     done = [torch.cuda.Event() for _ in range(nb)]
     out_free = [torch.cuda.Event() for _ in range(nb)]
 
-    def run_step(inp, o):
+    def run_step(inp, o, cs, wsi):
         if fused:
             pkv.paged_attn_decode_append(o, inp["q"], inp["k_new"], inp["v_new"], case.k_pool,
                                          case.v_pool, inp["block_tables"], inp["context_lens"],
                                          case.scale, mcl, partition_size=case.partition_size,
-                                         workspace=ws, err=err)
+                                         workspace=wsi, err=err, stream=cs)
             return
         pkv.kv_cache_append(case.k_pool, case.v_pool, inp["k_new"], inp["v_new"],
-                            inp["slot_mapping"], err=err)
+                            inp["slot_mapping"], err=err, stream=cs)
         pkv.paged_attn_decode(o, inp["q"], case.k_pool, case.v_pool, inp["block_tables"],
                               inp["context_lens"], case.scale, mcl,
-                              partition_size=case.partition_size, workspace=ws, err=err)
+                              partition_size=case.partition_size, workspace=wsi, err=err,
+                              stream=cs)
 
     def e2e_steps(n, start_event=None):
         for i in range(n):
@@ -650,22 +745,24 @@ def run_ours(args, rank, world, local_rank):
                     h2d_stream.wait_event(start_event)
                 dev_stage[b].copy_(host_stage, non_blocking=True)
                 in_ready[b].record(h2d_stream)
-            stream.wait_event(in_ready[b])
+            cs, wsi = comp[i % ncs], wss[i % ncs]
+            cs.wait_event(in_ready[b])
             if args.e2e_result_in_host_memory:
                 # the decode writes its result straight into pinned host memory
-                run_step(dev_sets[b], host_outs[b])
-                done[b].record(stream)
+                run_step(dev_sets[b], host_outs[b], cs, wsi)
+                done[b].record(cs)
                 out_free[b] = done[b]
                 continue
-            run_step(dev_sets[b], outs[b])
-            done[b].record(stream)
+            run_step(dev_sets[b], outs[b], cs, wsi)
+            done[b].record(cs)
             with torch.cuda.stream(d2h_stream):
                 d2h_stream.wait_event(done[b])
                 host_outs[b].copy_(outs[b], non_blocking=True)
                 out_free[b].record(d2h_stream)
-        last = torch.cuda.Event()
-        last.record(d2h_stream)
-        stream.wait_event(last)
+        for other in [d2h_stream] + comp[1:]:
+            last = torch.cuda.Event()
+            last.record(other)
+            stream.wait_event(last)
 
     e2e_steps(3)
     torch.cuda.synchronize()
@@ -706,8 +803,26 @@ def run_ours(args, rank, world, local_rank):
 
     swap = measure_swap(case, dev, stream, pkv) if args.workload != "shared_prefix" else None
 
+    # standalone kv_cache_append of the step's tokens (through the slot mapping)
+    append_line = None
+    if case.slot_mapping is not None and not args.no_extras:
+        for _ in range(3):
+            pkv.kv_cache_append(case.k_pool, case.v_pool, case.k_new, case.v_new,
+                                case.slot_mapping, err=err)
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a_ev.record(stream)
+        for _ in range(args.steps):
+            pkv.kv_cache_append(case.k_pool, case.v_pool, case.k_new, case.v_new,
+                                case.slot_mapping, err=err)
+        b_ev.record(stream)
+        torch.cuda.synchronize()
+        app_ms = a_ev.elapsed_time(b_ev) / args.steps
+        append_line = {"tokens": S, "us": app_ms * 1e3, "bytes": app_bytes,
+                       "GB/s": app_bytes / (app_ms * 1e-3) / 1e9}
+
     contiguous = None
-    if args.contiguous and args.workload != "shared_prefix":
+    if (args.contiguous or not args.no_extras) and args.workload != "shared_prefix":
         ccase = make_case(args.workload, device=dev, with_append=False, placement="identity",
                           num_seqs=args.num_seqs)
         cout = torch.empty_like(ccase.q)
@@ -730,10 +845,14 @@ def run_ours(args, rank, world, local_rank):
                       "paged_over_contiguous_time": sms / cms}
         del ccase, cout
 
+    peak, peak_kind = measured_peaks()
+    # every rank times the same extra workloads on its own GPU (no collective);
+    # rank 0 reports its own
+    extras_all = {} if args.no_extras else extra_lines(args, dev, rank, pkv, stream, peak)
+
     if rank != 0:
         return None
 
-    peak, peak_kind = measured_peaks()
     # the fused call also reads the new K/V rows and writes them to the pool
     call_bytes = dec_bytes + (app_bytes if fused else 0)
     achieved = call_bytes / (dec_ms * 1e-3) / 1e9
@@ -761,7 +880,8 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "pipelining": "inputs staged in one pinned buffer, one upload per step on a copy "
-                              "stream, overlapping the neighbouring steps' kernels",
+                              "stream, overlapping the neighbouring steps' kernels; steps take "
+                              f"turns on {ncs} compute stream(s), each with its own workspace",
                 "result_to_host": ("written by the decode kernels into pinned host memory"
                                    if args.e2e_result_in_host_memory else
                                    "device-to-host copy on a second copy stream"),
@@ -774,19 +894,22 @@ def run_ours(args, rank, world, local_rank):
     }
     if contiguous:
         line["paged_vs_contiguous"] = contiguous
+    if append_line:
+        line["kv_cache_append"] = append_line
+    line.update(extras_all)
     if swap:
         swap["pinned_h2d_gbs"], swap["pinned_d2h_gbs"] = h2d_gbs, d2h_gbs
         line["swap"] = swap
-    line["config"]["call"] = ("kv_cache_append + paged_attn_decode" if not fused else
-                              "paged_attn_decode_append (append fused into the decode)")
+    line["config"]["call"] = call_description(case, args)
     line.update(extras)
-    for key in ("beam_search", "prefix_cache"):
+    for key in ("shared_prefix", "beam_search", "prefix_cache"):
         if key in extras:
+            # the unique step: each distinct block's K/V once, plus the q/o,
+            # table and append bytes of every sequence
             bx = extras[key]
-            bx["unique_gbs"] = bx["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
-    if "shared_prefix" in extras:
-        sp_x = extras["shared_prefix"]
-        sp_x["unique_gbs"] = sp_x["unique_kv_bytes"] / (dec_ms * 1e-3) / 1e9
+            bx["unique_bytes"] = bx["unique_kv_bytes"] + (call_bytes - bx["logical_kv_bytes"])
+            bx["unique_GB/s"] = bx["unique_bytes"] / (dec_ms * 1e-3) / 1e9
+            bx["unique_frac"] = bx["unique_GB/s"] / peak
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, args.cpu_seconds)
     return line

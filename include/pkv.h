@@ -75,11 +75,14 @@ enum {
 
 /*
  * Bytes of device workspace paged_attn_decode needs for these sizes: a few
- * scheduling words and the work list (one 8-byte entry per possible
- * (sequence, partition) pair), plus, when a context can span several
- * partitions, one fp32 output row and one fp32 log-sum-exp per (sequence,
- * query head, partition). Always > 0 for num_seqs > 0. This function is pure
- * arithmetic: it does not touch the GPU.
+ * scheduling words, the work list (one 8-byte entry per possible
+ * (sequence, partition) pair), two int32 per sequence for the shared-prefix
+ * grouping, merge counters, and R fp32 output rows plus R fp32 log-sum-exp
+ * values per (sequence, query head), where R is the partition count of a
+ * max_context_len context, and at least 2 (the work of sequences that share
+ * a prefix may be split in two even when no single context needs a split).
+ * Always > 0 for num_seqs > 0. This function is pure arithmetic: it does not
+ * touch the GPU.
  */
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_context_len, int partition_size);
@@ -127,6 +130,13 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  * Long contexts are split into partitions of partition_size tokens. Each
  * partition is attended independently, and the partials are combined by
  * log-sum-exp weights.
+ *
+ * Sequences next to each other in the batch whose block tables start with the
+ * same physical blocks (forked samples, beams, cached prefixes: page
+ * "PagedAttention Analysis", section 4) are attended together when
+ * num_heads / num_kv_heads is 1 or 2: the whole 16-token tiles of their common
+ * leading blocks are read once for all of them. Each sequence still gets its
+ * own attention over its own tokens; only the fp32 summation order differs.
  *
  * out            [num_seqs][num_heads][head_dim], written entirely. A sequence
  *                with L <= 0 gets zeros. Device memory, or page-locked host
@@ -190,7 +200,11 @@ int paged_attn_decode(void *out, const void *q, const void *k_pool, const void *
  *    until the process exits.
  *  - The first call on a device looks up that copy's address (one
  *    cudaGetSymbolAddress) with the device current. Make that first call
- *    before any stream capture.
+ *    before any stream capture. The address is kept per device together
+ *    with the id of the context it belongs to; after a cudaDeviceReset the
+ *    next call sees a new context and looks the address up again.
+ *  - num_seqs <= 0 needs no workspace: the call then returns what
+ *    paged_attn_decode returns for the same arguments.
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents; the decode resets what it needs on every call. Calls whose
  *    GPU work can overlap in time (different streams without ordering between

@@ -68,6 +68,8 @@
 // Every wait is bounded: one that gives up sets an error status and a
 // CTA-wide stop flag, and the kernel winds down, first waiting (bounded) for
 // the copies it still has in flight.
+#include <climits>
+
 #include "pkv_device.cuh"
 #include "pkv_internal.h"
 
@@ -103,15 +105,29 @@ constexpr int KIND_NOP = 3;          // keeps the ring turning while the last it
 constexpr int KIND_END = 4;          // no more descriptors
 constexpr int PLAN_BUCKETS = 64;     // size classes for ordering the short last partitions
 
-// One entry of the scheduler -> consumer descriptor ring.
-struct ItemDesc {
-  int kind, s, p, h, L, n_tiles, nparts;
-  int new_tok;  // fused append: partition-relative index of token L-1, or -1
-  int ids[DESC_IDS];    // physical block of tile (or 8-token unit) t; -1 past the context
+// Most sequences one work item attends together (a shared-prefix group).
+constexpr int MAX_MEMBERS = 8;
+
+// One entry of the scheduler -> consumer descriptor ring. A work item attends
+// `members` sequences s, s+1, ... (one, or a group that shares its first `sh`
+// tiles) for one KV head. Its tiles are numbered group-wide: the shared tiles
+// 0 .. sh-1 (tokens 0 .. 16*sh-1 of every member), then member m's own tiles
+// own[m] .. own[m+1]-1 (its tokens from 16*sh on). Partition p covers group
+// tiles tile0 .. tile0 + n_tiles - 1.
+struct alignas(16) ItemDesc {
+  int kind, s, p, h, n_tiles, nparts;
+  int members;   // sequences attended by this item
+  int tile0;     // group tile of the partition's first tile
+  int sh;        // shared tiles (0 for one sequence)
+  int own[MAX_MEMBERS + 1];  // first own tile of each member; own[members] = all tiles
+  int len[MAX_MEMBERS];      // members' context lengths
+  int ids[DESC_IDS];  // physical block of tile (or 8-token unit) t; -1 past the context
 };
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base). NH is
-// the number of head rows an instantiation carries (4 or 8 >= G).
+// the number of score columns (query-head rows) an item carries: the G heads
+// of one sequence (NH = 4 serves G = 3, 4), or with NH = 8 the heads of up to
+// 8 / G sequences that share a prefix (G = 1, 2; one sequence for G = 5..8).
 template <int D, int NH>
 struct TcShape {
   static constexpr int HALVES = D / BOX_COLS;
@@ -119,25 +135,40 @@ struct TcShape {
   static constexpr int STAGE_BYTES = 2 * KT_BYTES;       // K + V
   static constexpr int ACC_STRIDE = D + 4;               // padded combine row (floats)
   static constexpr int CW_FLOATS = NH * ACC_STRIDE + 2 * NH;  // acc[NH][D+4], m[NH], l[NH]
-  static constexpr int COMBINE_BYTES = (NCW * CW_FLOATS + NH * (NCW + 1)) * 4;  // + scales
-  // per slot: the group's q rows, then the newest token's K and V rows (fused append)
-  static constexpr int QROWS_BYTES = NH * D * 2;
-  static constexpr int QBUF_BYTES = QROWS_BYTES + 2 * D * 2;
-  static constexpr int FIXED = COMBINE_BYTES + NSLOT * QBUF_BYTES +
-                               NSLOT * (int)sizeof(ItemDesc) + 64 * 8 + 1024 + 64;
+  // With 8 columns a warp's partial result of an item is combined from the
+  // ring stage of its last tile, which it refills only after the next item's
+  // vote: a combine area of its own (4 x 8 x 132 floats) would leave room for
+  // two stages only. With 4 columns the area fits beside three stages, and a
+  // warp refills its last stage at once.
+  static constexpr bool RING_COMBINE = NH >= 8;
+  static_assert(!RING_COMBINE || CW_FLOATS * 4 <= STAGE_BYTES, "a stage holds the rows");
+  static constexpr int COMBINE_BYTES = RING_COMBINE ? 0 : NCW * CW_FLOATS * 4;
+  // weights [NH][NCW], log2-sum-exp [NH], each warp's combine stage [NCW]
+  static constexpr int SCALES_BYTES = (NH * (NCW + 1) + NCW) * 4;
+  // One sequence per item (4 columns): its newest K and V rows travel with
+  // its q rows; groups (8 columns) read them from k_new / v_new.
+  static constexpr bool STAGED_NEW = !RING_COMBINE;
+  static constexpr int QROWS_BYTES = NH * D * 2;  // the q rows of every member
+  static constexpr int QBUF_BYTES = QROWS_BYTES + (STAGED_NEW ? 2 * D * 2 : 0);
+  static constexpr int FIXED = COMBINE_BYTES + ((SCALES_BYTES + 15) & ~15) +
+                               NSLOT * QBUF_BYTES + NSLOT * (int)sizeof(ItemDesc) + 64 * 8 +
+                               1024 + 64;
   // As many stages as fit two CTAs per SM, at most 6. An SM has 228 KB of
   // shared memory and each CTA also reserves 1 KB, so a CTA may use ~113 KB.
   static constexpr int CTA_SMEM_BUDGET = 228 * 1024 / 2 - 1024 - 256;
   static constexpr int NSTAGE_FIT = (CTA_SMEM_BUDGET - FIXED) / (NCW * STAGE_BYTES);
   static constexpr int NSTAGE = NSTAGE_FIT > 6 ? 6 : NSTAGE_FIT;
-  static_assert(NSTAGE >= 2, "ring too shallow");
+  static_assert(NSTAGE >= 3, "ring too shallow");
   static constexpr int RING_BYTES = NCW * NSTAGE * STAGE_BYTES;
   static constexpr int COMBINE_OFF = RING_BYTES;
-  static constexpr int QBUF_OFF = COMBINE_OFF + ((COMBINE_BYTES + 15) & ~15);
+  static constexpr int SCALES_OFF = COMBINE_OFF + COMBINE_BYTES;
+  static constexpr int QBUF_OFF = SCALES_OFF + ((SCALES_BYTES + 15) & ~15);
   static constexpr int DESC_OFF = QBUF_OFF + NSLOT * QBUF_BYTES;
   static constexpr int BAR_OFF = DESC_OFF + NSLOT * (int)sizeof(ItemDesc);
   static constexpr int NBARS = NCW * NSTAGE + 2 * NSLOT;
+  static_assert(NBARS <= 64, "barrier area");
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= CTA_SMEM_BUDGET, "two CTAs per SM");
   static_assert(QBUF_OFF % 16 == 0 && DESC_OFF % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
 };
 
@@ -145,21 +176,171 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
   return (static_cast<uint32_t>(s) << 16) | static_cast<uint32_t>(p);
 }
 
+// Tiles per partition of an entry. One sequence uses the call's partition
+// length. A group of sequences that share a prefix (see plan_groups) spans its
+// shared tiles once plus every member's own tiles; it is cut into balanced
+// partitions of at most GROUP_PART_TILES tiles (or the call's length, if
+// shorter), as many as the workspace rows each member has (max_parts) allow,
+// so that a few large group items do not leave most CTAs idle at the end.
+constexpr int GROUP_PART_TILES = 64;
+__device__ __forceinline__ int group_part_tiles(const DecodeArgs &a, bool grouped, int tiles) {
+  const int pt = a.part_tokens / TILE;
+  if (!grouped) return pt;
+  const int want = min(pt, GROUP_PART_TILES);
+  const int np = max(1, min(a.max_parts, (tiles + want - 1) / want));
+  return max(1, (tiles + np - 1) / np);
+}
+
+// Inclusive prefix maximum over the plan block (one value per thread).
+__device__ __forceinline__ int plan_block_max_scan(int v, int *wmax) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(FULL_MASK, v, off);
+    if (lane >= off) v = max(v, y);
+  }
+  if (lane == 31) wmax[warp] = v;
+  __syncthreads();
+  int before = INT_MIN;
+  for (int w = 0; w < warp; ++w) before = max(before, wmax[w]);
+  __syncthreads();  // wmax is reused by the next scan
+  return max(v, before);
+}
+
+// Shared-prefix groups, found by the plan kernel when a.max_group > 1.
+//
+// Sequences that share blocks (the samples of one prompt, the beams of one
+// request, requests that hit the same cached prefix: page "PagedAttention
+// Analysis", section 4, and the copy-on-write section of page "추론 엔진에서의
+// 메모리 가상화") point to the same physical blocks from the start of their
+// block tables. A physical block holds one set of K/V values whoever reads it,
+// so adjacent sequences whose table entries agree up to some block can be
+// attended by one work item that reads those shared tiles once, with every
+// member's query rows side by side in the tensor-core N dimension.
+//
+// For each round of PLAN_THREADS sequences:
+//  - psh(s): the tiles of 16 tokens that sequence s shares with s-1: the
+//    tokens of all blocks before the first table entry where they differ,
+//    capped at both lengths and rounded down to whole tiles. With a fused
+//    append each sequence's newest token is excluded (it is written in this
+//    call, so it is never read as shared).
+//  - A run is a maximal stretch of sequences each sharing at least one tile
+//    with its predecessor; runs do not cross rounds. A run is cut into groups
+//    of at most a.max_group members, and a group's shared length is the
+//    smallest psh inside it.
+//  - a.grp[s] = 0 for a sequence on its own, (members - 1) << 27 | shared
+//    tiles for a group's first member (its leader), -1 for the other members;
+//    a.grp_tiles[leader] = shared tiles + every member's own tiles.
+// The table comparison touches only candidate pairs (equal first entries) and
+// only the entries that both sequences' shared span covers, spread over all
+// threads of the block.
+// Returns whether any group formed (uniform over the block); when none did,
+// a.grp is not written and the caller treats every sequence as its own.
+template <typename EffLen, typename BlockScan>
+__device__ __noinline__ bool plan_groups(const DecodeArgs &a, EffLen eff_len,
+                                         BlockScan block_scan) {
+  __shared__ int c_seq[PLAN_THREADS];     // candidate pairs (s-1, s): s
+  __shared__ int c_off[PLAN_THREADS];     // first comparison index of each candidate
+  __shared__ int c_mis[PLAN_THREADS];     // first differing block (or the blocks compared)
+  __shared__ int g_cnt[PLAN_THREADS];     // members of the group a thread leads
+  __shared__ int g_sh[PLAN_THREADS];      // its shared tiles
+  __shared__ int g_own[PLAN_THREADS];     // its members' own tiles
+  __shared__ int wmax[PLAN_THREADS / 32];
+  const int tid = threadIdx.x;
+  const int S = a.num_seqs, B = a.block_size;
+  const int newest = a.k_new != nullptr ? 1 : 0;
+  bool any = false;
+  for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
+    const int s = r0 + tid;
+    const int L = s < S ? eff_len(s) : 0;
+    int cap = 0;  // tiles the pair (s-1, s) could share
+    bool cand = false;
+    if (s < S && tid > 0) {
+      // (the first entries are loaded with the lengths; they count only if cap > 0)
+      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
+      const int32_t b_this = bt[0], b_prev = (bt - a.max_blocks)[0];  // row s-1 precedes row s
+      cap = (min(L, eff_len(s - 1)) - newest) / TILE;
+      cand = cap > 0 && b_this == b_prev;
+    }
+    const int nblk = cand ? (cap * TILE + B - 1) / B : 0;  // blocks covering the span
+    int ncand, work;
+    const int ci = block_scan(cand ? 1 : 0, ncand);
+    if (ncand == 0) {  // (uniform) no pair of this round starts with the same block
+      if (any && s < S) a.grp[s] = 0;
+      continue;
+    }
+    if (!any) {  // the earlier rounds had no group: record them as single sequences
+      for (int i = tid; i < r0; i += PLAN_THREADS) a.grp[i] = 0;
+      any = true;
+    }
+    const int co = block_scan(cand ? nblk - 1 : 0, work);  // block 0 is already compared
+    if (cand) {
+      c_seq[ci] = s;
+      c_off[ci] = co;
+      c_mis[ci] = nblk;
+    }
+    g_cnt[tid] = 0;
+    g_sh[tid] = INT_MAX;
+    g_own[tid] = 0;
+    __syncthreads();
+    // every comparison of every candidate: f -> (candidate c, block j >= 1)
+    for (int f = tid; f < work; f += PLAN_THREADS) {
+      int lo = 0, hi = ncand - 1;  // the last candidate whose range starts at or before f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (c_off[mid] <= f)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      const int j = f - c_off[lo] + 1;
+      if (j < *static_cast<volatile int *>(&c_mis[lo])) {  // skip past a known difference
+        const int32_t *bt = a.block_tables + (size_t)c_seq[lo] * a.max_blocks;
+        if (bt[j] != (bt - a.max_blocks)[j]) atomicMin(&c_mis[lo], j);
+      }
+    }
+    __syncthreads();
+    const int psh = cand ? min(c_mis[ci] * B / TILE, cap) : 0;
+    const bool linked = psh > 0;  // never for tid 0: runs do not cross rounds
+    const int run = plan_block_max_scan(linked ? -1 : tid, wmax);
+    const int lead = run + (tid - run) / a.max_group * a.max_group;
+    if (s < S) {
+      atomicAdd(&g_cnt[lead], 1);
+      if (tid != lead) atomicMin(&g_sh[lead], psh);
+    }
+    __syncthreads();
+    const int members = g_cnt[lead];
+    const int sh = members > 1 ? g_sh[lead] : 0;
+    if (s < S && members > 1) atomicAdd(&g_own[lead], (L - sh * TILE + TILE - 1) / TILE);
+    __syncthreads();
+    if (s < S) {
+      int word = 0;
+      if (members > 1) word = tid == lead ? ((members - 1) << 27) | sh : -1;
+      a.grp[s] = word;
+      if (word > 0) a.grp_tiles[s] = sh + g_own[lead];
+    }
+    __syncthreads();  // the shared arrays are rewritten by the next round
+  }
+  return any;
+}
+
 // Build the work list in two regions.
-//  1. Sequences that span several partitions: all their partitions, sequence
-//     by sequence, the short last partition first. Their merges then complete
-//     while the list is still being worked through.
-//  2. Sequences of one partition, ordered by size, largest first (a counting
+//  1. Entries of several partitions: all their partitions, entry by entry,
+//     the short last partition first. Their merges then complete while the
+//     list is still being worked through.
+//  2. Entries of one partition, ordered by size, largest first (a counting
 //     sort over PLAN_BUCKETS size classes). They need no merge, and handing out
 //     the largest first and the smallest last keeps the CTAs' finishing times
-//     close. The sort is stable: within a size class the sequences keep their
-//     order, so sequences that share blocks and sit next to each other in the
-//     batch (the samples of one prompt) are attended together, and their shared
-//     blocks are fetched once and then served from L2. A sequence of length 0 is
-//     one (empty) entry, so that its output is still written.
-// Each entry carries the sequence's clamped length. Sequences are taken in
-// rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t), so
-// that thread order is sequence order. The merge counters are reset here too.
+//     close. The sort is stable: within a size class the entries keep batch
+//     order. A sequence of length 0 is one (empty) entry, so that its output
+//     is still written.
+// An entry is one sequence, or, when a.max_group > 1, one group of adjacent
+// sequences that share their first blocks (plan_groups): the group's leader
+// carries it and the other members have no entry. Each entry carries the
+// sequence's clamped length, or the leader's group word. Sequences are taken
+// in rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t),
+// so that thread order is sequence order. The merge counters are reset here
+// too.
 //
 // This grid is the programmatic dependent of what precedes it, typically the
 // previous decode call, and may start while that call is still running. It
@@ -178,14 +359,14 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   pdl_wait();
   uint2 *const list = a.work;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int S = a.num_seqs, P = a.part_tokens;
+  const int S = a.num_seqs;
+  bool grouping = a.max_group > 1;
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
   if (tid == 0) bad_len = 0;
   __syncthreads();
-  const int max_tiles = max(1, P / 16);
-  // size class of a one-partition sequence of `len` tokens: bigger -> smaller class
-  auto bucket = [&](int len) {
-    const int tiles = (len + 15) / 16;
+  const int max_tiles = max(1, a.part_tokens / TILE);
+  // size class of a one-partition entry of `tiles` tiles: bigger -> smaller class
+  auto bucket = [&](int tiles) {
     return (PLAN_BUCKETS - 1) - min(PLAN_BUCKETS - 1, tiles * (PLAN_BUCKETS - 1) / max_tiles);
   };
   // Exclusive block-wide prefix sum of v; `total` receives the sum.
@@ -213,6 +394,30 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     __syncthreads();  // wsum is reused by the next scan
     return excl;
   };
+  auto eff_len = [&](int s) {
+    return effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, a.block_size,
+                         nullptr);
+  };
+
+  if (grouping) grouping = plan_groups(a, eff_len, block_scan);
+
+  // Tiles and partitions of sequence s's entry (np = 0: no entry; a group
+  // member other than the leader). `word` is the entry's second field.
+  auto entry_shape = [&](int s, int L, int &np, int &tiles, uint32_t &word) {
+    const int g = grouping ? a.grp[s] : 0;
+    word = (uint32_t)L;
+    tiles = (L + TILE - 1) / TILE;
+    if (g < 0) {
+      np = 0;
+      return;
+    }
+    if (g > 0) {
+      tiles = a.grp_tiles[s];
+      word = 0x80000000u | (uint32_t)g;
+    }
+    const int ptg = group_part_tiles(a, g > 0, tiles);
+    np = max(1, (tiles + ptg - 1) / ptg);  // an empty sequence still has its (empty) entry
+  };
 
   // pass 1: region-1 entry count and the size-class histogram of region 2
   int nm = 0;
@@ -220,12 +425,15 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     const int s = r0 + tid;
     if (s < S) {
       const int raw = a.context_lens[s];
-      const int L = effective_len(raw, a.max_context_len, a.max_blocks, a.block_size, nullptr);
+      const int L = eff_len(s);
       if (L < raw) bad_len = 1;
-      if (L > P)
-        nm += (L + P - 1) / P;
-      else
-        atomicAdd(&hist[bucket(L)], 1);
+      int np, tiles;
+      uint32_t word;
+      entry_shape(s, L, np, tiles, word);
+      if (np > 1)
+        nm += np;
+      else if (np == 1)
+        atomicAdd(&hist[bucket(tiles)], 1);
     }
   }
   int total_m;
@@ -250,21 +458,22 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   // pass 2: write the entries, one round of PLAN_THREADS sequences at a time
   for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
     const int s = r0 + tid;
-    int L = 0, np = 0, bkt = -1;
+    int np = 0, bkt = -1;
+    uint32_t word = 0;
     if (s < S) {
-      L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, a.block_size,
-                        nullptr);
-      if (L > P)
-        np = (L + P - 1) / P;
-      else
-        bkt = bucket(L);
+      int n, tiles;
+      entry_shape(s, eff_len(s), n, tiles, word);
+      if (n > 1)
+        np = n;
+      else if (n == 1)
+        bkt = bucket(tiles);
     }
     // region 1: this round's entries after the previous rounds'
     int round_m;
     const int om = total_m_s + block_scan(np, round_m);
     if (np > 0) {
-      list[om] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
-      for (int q = 0; q < np - 1; ++q) list[om + 1 + q] = make_uint2(pack_pair(s, q), (uint32_t)L);
+      list[om] = make_uint2(pack_pair(s, np - 1), word);
+      for (int q = 0; q < np - 1; ++q) list[om + 1 + q] = make_uint2(pack_pair(s, q), word);
     }
     // region 2: rank among this warp's lanes of the same class, then the
     // earlier warps' counts, then the class's running start
@@ -285,7 +494,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     }
     if (tid == 0) total_m_s += round_m;
     __syncthreads();
-    if (bkt >= 0) list[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+    if (bkt >= 0) list[wcnt[warp][bkt] + rank] = make_uint2(pack_pair(s, 0), word);
     __syncthreads();  // wcnt and total_m_s are rewritten by the next round
   }
   const int total = total_s;
@@ -408,23 +617,25 @@ __device__ __forceinline__ bool consumers_all(bool v) {
   return r != 0;
 }
 
-// Merge entries [q0, q1) (at most MERGE_CHUNK) of one (sequence, KV head):
-// for each of its G query heads, o = sum_q 2^(lse_q - lse) o_q with
-// lse = log2 sum_q 2^lse_q. The sources were written by other CTAs; they are
-// read from L2 (ld.global.cg). The result goes to `out` (final), or to chunk
-// entry `dst_idx` of the second-level arrays as (o, lse).
+// Merge entries [q0, q1) (at most MERGE_CHUNK) of one work item's KV head,
+// for the G query heads of each of its `members` sequences s, s+1, ...:
+// o = sum_q 2^(lse_q - lse) o_q with lse = log2 sum_q 2^lse_q. The sources
+// were written by other CTAs; they are read from L2 (ld.global.cg). The
+// result goes to `out` (final), or to chunk entry `dst_idx` of the
+// second-level arrays as (o, lse).
 template <typename T, int D>
-__device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int G,
+__device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int G, int members,
                                          const float *src_o, const float *src_lse,
                                          int src_stride, int q0, int q1, bool final_out,
                                          int dst_idx) {
   constexpr int V = D / 4;  // float4 columns per head row
   T *const out = static_cast<T *>(a.out);
   const int n_q = q1 - q0;
-  for (int idx = threadIdx.x; idx < G * V; idx += NCW * 32) {
+  for (int idx = threadIdx.x; idx < members * G * V; idx += NCW * 32) {
     const int n = idx / V;
     const int cv = idx - n * V;
-    const size_t row = (size_t)s * a.num_heads + h * G + n;
+    const int mem = n / G;
+    const size_t row = (size_t)(s + mem) * a.num_heads + h * G + (n - mem * G);
     const float *lse = src_lse + row * src_stride + q0;
     const float4 *po = reinterpret_cast<const float4 *>(src_o + (row * src_stride + q0) * D) + cv;
     float M = -INFINITY;
@@ -460,6 +671,42 @@ __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int 
       if (cv == 0) a.ws2_lse[row * a.max_chunks + dst_idx] = W > 0.f ? M + log2f(W) : -INFINITY;
     }
   }
+}
+
+// Where group tile gt of a work item lies: in the shared span (m = -1; every
+// member's tokens, all valid, read through the first member's table), or in
+// member m's own span (its tokens from 16*sh on). tok0 is the tile's first
+// token in that sequence; len bounds the valid tokens.
+struct TileLoc {
+  int m, tok0, len;
+};
+
+// A warp's register copy of an item's layout: lane i < members holds member
+// i's first own tile and length (the lookup below then needs no shared-memory
+// reads per tile).
+struct ItemView {
+  int members, sh, len0, own_r, len_r;
+};
+__device__ __forceinline__ ItemView item_view(const ItemDesc &d, int lane) {
+  ItemView v;
+  v.members = d.members;
+  v.sh = d.sh;
+  v.len0 = d.len[0];
+  v.own_r = lane < v.members ? d.own[lane] : INT_MAX;
+  v.len_r = lane < v.members ? d.len[lane] : 0;
+  return v;
+}
+
+// Called by all lanes of a warp with the same gt.
+__device__ __forceinline__ TileLoc locate_tile(const ItemView &v, int gt, int lane) {
+  if (v.members == 1) return TileLoc{0, gt * TILE, v.len0};  // one sequence: all its own
+  if (gt < v.sh) return TileLoc{-1, gt * TILE, INT_MAX};
+  // own[] is non-decreasing: the member is the number of later members that
+  // start at or before gt (lanes past the members hold INT_MAX)
+  const int m = __popc(__ballot_sync(FULL_MASK, lane >= 1 && v.own_r <= gt));
+  const int own = __shfl_sync(FULL_MASK, v.own_r, m);
+  const int len = __shfl_sync(FULL_MASK, v.len_r, m);
+  return TileLoc{m, (v.sh + gt - own) * TILE, len};
 }
 
 // U8: the block size is an odd multiple of 8, so a 16-token tile is two
@@ -528,7 +775,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (;; ++it) {
       const int slot = it % NSLOT;
       ItemDesc &d = desc[slot];
-      int merge_kind = -1, merge_s = 0, merge_h = 0, merge_np = 0, merge_p = 0;
+      int merge_kind = -1, merge_s = 0, merge_h = 0, merge_np = 0, merge_p = 0, merge_m = 1;
       if (it >= NSLOT) {
         if (!__all_sync(FULL_MASK, wait_or_abort(item_empty(slot), ((it / NSLOT) - 1) & 1,
                                                  abort_flag, a.err)))
@@ -562,6 +809,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           merge_s = d.s;
           merge_h = d.h;
           merge_np = np;
+          merge_m = d.members;
           merge_p = __shfl_sync(FULL_MASK, next_p, 0);
         }
       }
@@ -573,6 +821,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           d.h = merge_h;
           d.p = merge_p;
           d.nparts = merge_np;
+          d.members = merge_m;
           d.n_tiles = 0;
           mbar_arrive(item_full(slot));
         }
@@ -616,13 +865,32 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int h = item - (item / Hkv) * Hkv;
       const int s = min(static_cast<int>(wk.x >> 16), a.num_seqs - 1);
       const int p = static_cast<int>(wk.x & 0xffffu);
-      const int L = static_cast<int>(wk.y);  // clamped (and checked) by the plan
-      const int t_begin = p * a.part_tokens;
-      const int t_end = min(L, t_begin + a.part_tokens);
-      const int n_tiles = t_end > t_begin ? (t_end - t_begin + TILE - 1) / TILE : 0;
-      // Fused append: the partition holding token L-1 also stages that
-      // token's new K and V rows.
-      const bool has_new = a.k_new != nullptr && n_tiles > 0 && t_end == L;
+      // One sequence (its clamped length in the entry), or a shared-prefix
+      // group led by s (its members' lengths are read here, clamped as the
+      // plan clamped them).
+      const bool grouped = (wk.y >> 31) != 0;
+      const int members =  // (the plan never forms more; the bounds keep every copy in place)
+          grouped ? min((int)((wk.y >> 27) & 15u) + 1,
+                        min(min(MAX_MEMBERS, max(1, NH / G)), a.num_seqs - s))
+                  : 1;
+      const int sh = grouped ? (int)(wk.y & 0x7ffffffu) : 0;
+      int Lm = 0;  // lane m < members: member m's length and own tiles
+      if (lane < members)
+        Lm = grouped ? effective_len(a.context_lens[s + lane], a.max_context_len, a.max_blocks, B,
+                                     nullptr)
+                     : static_cast<int>(wk.y);
+      const int own_n = lane < members ? max(0, Lm - sh * TILE + TILE - 1) / TILE : 0;
+      int own_incl = own_n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, own_incl, off);
+        if (lane >= off) own_incl += y;
+      }
+      const int own_lo = sh + own_incl - own_n;  // member lane's first own tile
+      const int tiles = sh + __shfl_sync(FULL_MASK, own_incl, 31);
+      const int ptg = group_part_tiles(a, grouped, tiles);
+      const int tile0 = p * ptg;
+      const int n_tiles = max(0, min(tiles, tile0 + ptg) - tile0);
       if (first_post) {
         first_post = false;
         if (__shfl_sync(FULL_MASK, err_word == PKV_DEV_WAIT_TIMEOUT ? 1 : 0, 0)) {
@@ -630,47 +898,96 @@ __global__ void __launch_bounds__(THREADS, 2)
           break;
         }
       }
-      // The group's q rows (and the new rows) are copied first: the copies
+      // The members' q rows (and, with one sequence per item, the newest
+      // token's K and V rows of a fused append) are copied first: the copies
       // complete on the slot's barrier while the lanes fetch the block ids,
       // and the arrival that publishes the descriptor comes last.
-      if (lane == 0) {
-        const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
-        const uint32_t rbytes = has_new ? (uint32_t)(D * 2) : 0u;
-        mbar_expect_tx(item_full(slot), qbytes + 2 * rbytes);
-        const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES;
-        if (qbytes)
-          bulk_load(stage, static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
-                    item_full(slot));
-        if (rbytes) {
-          const size_t row = ((size_t)s * Hkv + h) * D;
-          bulk_load(stage + Shape::QROWS_BYTES, static_cast<const T *>(a.k_new) + row, rbytes,
-                    item_full(slot));
-          bulk_load(stage + Shape::QROWS_BYTES + D * 2, static_cast<const T *>(a.v_new) + row,
-                    rbytes, item_full(slot));
+      const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
+      const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES;
+      if constexpr (Shape::STAGED_NEW) {  // one sequence: lane 0 issues everything
+        const int last = own_n - 1;       // its last tile holds token L-1
+        const uint32_t rbytes =
+            a.k_new != nullptr && last >= tile0 && last < tile0 + n_tiles ? (uint32_t)(D * 2) : 0u;
+        if (lane == 0) {
+          mbar_expect_tx(item_full(slot), qbytes + 2 * rbytes);
+          if (qbytes)
+            bulk_load(stage, static_cast<const T *>(a.q) + ((size_t)s * Hq + h * G) * D, qbytes,
+                      item_full(slot));
+          if (rbytes) {
+            const size_t row = ((size_t)s * Hkv + h) * D;
+            bulk_load(stage + Shape::QROWS_BYTES, static_cast<const T *>(a.k_new) + row, rbytes,
+                      item_full(slot));
+            bulk_load(stage + Shape::QROWS_BYTES + D * 2, static_cast<const T *>(a.v_new) + row,
+                      rbytes, item_full(slot));
+          }
         }
+      } else {
+        if (lane == 0) mbar_expect_tx(item_full(slot), members * qbytes);
+        __syncwarp();  // the expected bytes are set before any copy can complete
+        if (lane < members && qbytes)
+          bulk_load(stage + lane * qbytes,
+                    static_cast<const T *>(a.q) + ((size_t)(s + lane) * Hq + h * G) * D, qbytes,
+                    item_full(slot));
       }
-      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
       constexpr int upt = U8 ? 2 : 1;  // table entries per tile
       // All of a lane's table loads are issued before its first store.
       int idv[IDS_PER_LANE];
+      if (members == 1) {  // one sequence: partition tile t is its tile tile0 + t
+        const int L = __shfl_sync(FULL_MASK, Lm, 0);
+        const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
 #pragma unroll
-      for (int k = 0; k < IDS_PER_LANE; ++k) {
-        const int t = lane + 32 * k;
-        const int tok = t_begin + t * (TILE / upt);
-        idv[k] = t < n_tiles * upt && tok < L ? bt[tok / B] : -1;  // none read past the context
+        for (int k = 0; k < IDS_PER_LANE; ++k) {
+          const int t = lane + 32 * k;
+          const int tok = tile0 * TILE + t * (TILE / upt);
+          idv[k] = t < n_tiles * upt && tok < L ? bt[tok / B] : -1;  // none read past the context
+        }
+      } else {
+        // Member m's first own tile and length in every lane (for the lookup).
+        int own_v[MAX_MEMBERS], len_v[MAX_MEMBERS];
+#pragma unroll
+        for (int m = 0; m < MAX_MEMBERS; ++m) {
+          own_v[m] = __shfl_sync(FULL_MASK, own_lo, m);
+          len_v[m] = __shfl_sync(FULL_MASK, Lm, m);
+        }
+#pragma unroll
+        for (int k = 0; k < IDS_PER_LANE; ++k) {
+          const int t = lane + 32 * k;
+          const int gt = tile0 + t / upt;  // group tile
+          int m = 0, first = own_v[0], len = len_v[0];  // (selected without dynamic indexing)
+          if (gt >= sh) {  // a member's own tile
+#pragma unroll
+            for (int i = 1; i < MAX_MEMBERS; ++i)
+              if (i < members && own_v[i] <= gt) {
+                m = i;
+                first = own_v[i];
+                len = len_v[i];
+              }
+          }
+          const int tok = (gt >= sh ? sh + gt - first : gt) * TILE + (t % upt) * (TILE / upt);
+          // none read past the context
+          idv[k] = t < n_tiles * upt && tok < len
+                       ? a.block_tables[(size_t)(s + m) * a.max_blocks + tok / B]
+                       : -1;
+        }
       }
 #pragma unroll
       for (int k = 0; k < IDS_PER_LANE; ++k)
         if (lane + 32 * k < n_tiles * upt) d.ids[lane + 32 * k] = idv[k];
+      if (lane < members) {
+        d.own[lane] = own_lo;
+        d.len[lane] = Lm;
+      }
       if (lane == 0) {
         d.kind = KIND_WORK;
         d.s = s;
         d.p = p;
         d.h = h;
-        d.L = L;
         d.n_tiles = n_tiles;
-        d.nparts = (L + a.part_tokens - 1) / a.part_tokens;
-        d.new_tok = has_new ? L - 1 - t_begin : -1;
+        d.nparts = (tiles + ptg - 1) / ptg;
+        d.members = members;
+        d.tile0 = tile0;
+        d.sh = sh;
+        d.own[members] = tiles;
       }
       __syncwarp();  // every lane's ids precede lane 0's release below
       if (lane == 0) mbar_arrive(item_full(slot));
@@ -694,6 +1011,8 @@ __global__ void __launch_bounds__(THREADS, 2)
   // ======================= consumer warps =======================
   const int g = lane >> 2;  // mma group id (row of A / column of B)
   const int c = lane & 3;   // thread in group
+  // Members owning this lane's score columns 2c, 2c+1 (column n is member n / G).
+  const int mc0 = (2 * c) / G, mc1 = (2 * c + 1) / G;
   const float sl2 = a.scale_log2;
   T *const out = static_cast<T *>(a.out);
   const int mi = lane >> 3;                      // ldmatrix: lane feeds row (lane & 7)
@@ -701,16 +1020,18 @@ __global__ void __launch_bounds__(THREADS, 2)
   constexpr int AS = Shape::ACC_STRIDE;
   const uint32_t ring = smem0 + warp * NSTAGE * Shape::STAGE_BYTES;
   const int total_rows = a.num_blocks * Hkv * B;
-  float *const comb = reinterpret_cast<float *>(sm + Shape::COMBINE_OFF);
-  float *const cw_me = comb + warp * Shape::CW_FLOATS;  // this warp's combine rows
-  float *const scales = comb + NCW * Shape::CW_FLOATS;  // [NH][NCW] weights, [NH] lse
+  float *const scales = reinterpret_cast<float *>(sm + Shape::SCALES_OFF);  // [NH][NCW], [NH]
+  int *const comb_stage = reinterpret_cast<int *>(scales + NH * (NCW + 1));  // [NCW]
+  constexpr int CH = D / 8;                 // 16-byte chunks per K or V row
+  const int e_ch = lane % CH, kv_ch = lane / CH;  // fused append: lanes < CH K, < 2CH V
 
   // Issue side of this warp's ring. It walks the same descriptor sequence as
   // the consume side but runs up to NSTAGE tiles ahead, across item boundaries.
   uint32_t issued = 0, done = 0;  // tiles of this warp issued / consumed so far
   uint32_t bad_mask = 0;          // bit st: the tile in stage st had an invalid block id
   uint32_t is_it = 0;             // descriptor being issued
-  int is_j = 0, is_ntw = 0, is_h = 0, is_tbegin = 0, is_s = 0, is_L = 0;
+  int is_j = 0, is_ntw = 0, is_h = 0, is_tile0 = 0, is_s = 0;
+  ItemView is_view{1, 0, 0, 0, 0};
   bool is_ready = false, is_end = false;
 
   // Issue this warp's next tiles while fewer than NSTAGE are in flight. With
@@ -733,9 +1054,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
         const int nt = d.kind == KIND_WORK ? d.n_tiles : 0;
         is_s = d.s;
-        is_L = d.L;
         is_h = d.h;
-        is_tbegin = d.p * a.part_tokens;
+        is_tile0 = d.tile0;
+        is_view = item_view(d, lane);
         is_ntw = warp < nt ? (nt - warp + NCW - 1) / NCW : 0;
         is_j = 0;
         is_ready = true;
@@ -746,24 +1067,25 @@ __global__ void __launch_bounds__(THREADS, 2)
         continue;
       }
       const int tile = warp + is_j * NCW;
-      const int tok0 = is_tbegin + tile * TILE;
+      const ItemDesc &dd = desc[is_it % NSLOT];
+      const TileLoc loc = locate_tile(is_view, is_tile0 + tile, lane);
+      const int tok0 = loc.tok0;
+      const size_t trow = (size_t)(is_s + max(loc.m, 0)) * a.max_blocks;  // its table row
       const int st = issued % NSTAGE;
       // Pool row of each unit of the tile. total_rows is wholly out of
       // bounds, and TMA fills zeros there. It is used for an invalid block id,
       // which is reported, and for a second unit past the context, whose
-      // table entry is not read. The first unit always starts before L.
+      // table entry is not read. The first unit always starts before the end
+      // of its sequence.
       constexpr int upt = U8 ? 2 : 1;
       const int idx0 = tile * upt;
-      const int p0 = idx0 < DESC_IDS ? desc[is_it % NSLOT].ids[idx0]
-                                     : a.block_tables[(size_t)is_s * a.max_blocks + tok0 / B];
+      const int p0 = idx0 < DESC_IDS ? dd.ids[idx0] : a.block_tables[trow + tok0 / B];
       bool bad = p0 < 0 || p0 >= a.num_blocks;
       const int y0 = bad ? total_rows : (p0 * Hkv + is_h) * B + (tok0 % B);
       int y1 = total_rows;
-      if (U8 && tok0 + TILE / 2 < is_L) {
+      if (U8 && tok0 + TILE / 2 < loc.len) {
         const int tok1 = tok0 + TILE / 2;
-        const int p1 = idx0 + 1 < DESC_IDS
-                           ? desc[is_it % NSLOT].ids[idx0 + 1]
-                           : a.block_tables[(size_t)is_s * a.max_blocks + tok1 / B];
+        const int p1 = idx0 + 1 < DESC_IDS ? dd.ids[idx0 + 1] : a.block_tables[trow + tok1 / B];
         const bool bad1 = p1 < 0 || p1 >= a.num_blocks;
         bad = bad || bad1;
         if (!bad1) y1 = (p1 * Hkv + is_h) * B + (tok1 % B);
@@ -813,24 +1135,28 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int np = dref.nparts;
       if (kind == KIND_MERGE_CHUNK) {
         const int q0 = dref.p * MERGE_CHUNK;
-        merge_range<T, D>(a, dref.s, dref.h, G, a.ws_o, a.ws_lse, a.max_parts, q0,
+        merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws_o, a.ws_lse, a.max_parts, q0,
                           min(np, q0 + MERGE_CHUNK), false, dref.p);
       } else if (kind == KIND_MERGE_FINAL) {
         if (np <= MERGE_CHUNK)
-          merge_range<T, D>(a, dref.s, dref.h, G, a.ws_o, a.ws_lse, a.max_parts, 0, np, true, 0);
+          merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws_o, a.ws_lse, a.max_parts,
+                            0, np, true, 0);
         else
-          merge_range<T, D>(a, dref.s, dref.h, G, a.ws2_o, a.ws2_lse, a.max_chunks, 0,
-                            (np + MERGE_CHUNK - 1) / MERGE_CHUNK, true, 0);
+          merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws2_o, a.ws2_lse,
+                            a.max_chunks, 0, (np + MERGE_CHUNK - 1) / MERGE_CHUNK, true, 0);
       }
       pump(false);
       consumers_sync();  // the descriptor is read by all before the slot is handed back
       if (lane == 0) mbar_arrive(item_empty(slot));
       continue;
     }
-    const int s = dref.s, p = dref.p, h = dref.h, L = dref.L, n_tiles = dref.n_tiles;
+    const int s = dref.s, p = dref.p, h = dref.h, n_tiles = dref.n_tiles;
     const int nparts = dref.nparts;
-    const int new_tok = dref.new_tok;
-    const int t_begin = p * a.part_tokens;
+    const int members = dref.members, tile0 = dref.tile0;
+    const bool one_seq = members == 1;
+    const int ncol = members * G;  // head rows attended: G per member
+    // this lane's two columns (query heads 2c, 2c+1 of the rows) belong to these members
+    const bool col0_live = mc0 < members, col1_live = mc1 < members;
     const int nt_w = warp < n_tiles ? (n_tiles - warp + NCW - 1) / NCW : 0;
 
     pump(false);  // top up the ring (this item, and beyond)
@@ -843,7 +1169,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         const int Lc = (j >> 1) * 8 + 2 * c + (j & 1);
-        qf[j] = (g < G && n_tiles > 0) ? lds128(qrow + Lc * 16) : make_uint4(0, 0, 0, 0);
+        qf[j] = (g < ncol && n_tiles > 0) ? lds128(qrow + Lc * 16) : make_uint4(0, 0, 0, 0);
       }
     }
 
@@ -853,8 +1179,42 @@ __global__ void __launch_bounds__(THREADS, 2)
     float m0 = -INFINITY, m1 = -INFINITY;  // reference max of heads 2c, 2c+1 (base-2 units)
     float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
     bool aborted = false;
+    int last_st = -1;  // with RING_COMBINE: the stage of this warp's last tile of the item
+
+    const ItemView view = item_view(dref, lane);
+    const int L0 = view.len0;  // one sequence: its length
+    // Fused append, one sequence: the j of this warp's tile that holds token L-1.
+    int j_new = -1;
+    if (a.k_new != nullptr && one_seq && L0 > 0) {
+      const int idx = (L0 - 1) / TILE - tile0;
+      if (idx >= 0 && idx < n_tiles && idx % NCW == warp) j_new = idx / NCW;
+    }
+    // Fused append, 8 columns: the K (lanes < CH) or V (lanes CH..2CH-1) row
+    // chunk of the newest token of the member whose last tile is this warp's
+    // j-th tile, read from k_new / v_new one tile before it is used.
+    auto fetch_newest = [&](int j) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (!Shape::STAGED_NEW) {
+        if (a.k_new == nullptr || j >= nt_w) return v;  // (uniform)
+        int m = 0;
+        if (one_seq) {
+          if (j != j_new) return v;
+        } else {
+          const TileLoc l = locate_tile(view, tile0 + warp + j * NCW, lane);
+          if (l.m < 0 || l.len - 1 >= l.tok0 + TILE) return v;
+          m = l.m;
+        }
+        if (lane >= 2 * CH) return v;
+        const T *src = static_cast<const T *>(kv_ch ? a.v_new : a.k_new) +
+                       ((size_t)(s + m) * Hkv + h) * D + e_ch * 8;
+        v = __ldg(reinterpret_cast<const uint4 *>(src));
+      }
+      return v;
+    };
+    uint4 newest = fetch_newest(0);
 
     for (int j = 0; j < nt_w; ++j) {
+      const uint4 newest_next = fetch_newest(j + 1);
       if (issued == done) pump(true);
       const int st = done % NSTAGE;
       if (issued == done ||
@@ -865,28 +1225,51 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       const uint32_t ks = ring + st * Shape::STAGE_BYTES;
       const uint32_t vs = ks + Shape::KT_BYTES;
-      const int tok0 = t_begin + (warp + j * NCW) * TILE;
-      const int valid = min(TILE, L - tok0);
-      const bool bad = (bad_mask >> st) & 1u;
-
       const int tile_idx = warp + j * NCW;
-      if (new_tok >= 0 && (new_tok >> 4) == tile_idx && !bad) {
-        // Fused append: this tile holds token L-1. Its K and V rows come from
-        // the staged new rows (whatever the pool slot held), and the same rows
-        // are written to the pool slot: that is the cache-append.
-        const int r = new_tok & (TILE - 1);
-        const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES +
-                               Shape::QROWS_BYTES;
-        constexpr int CH = D / 8;  // 16-byte chunks per row
-        const int e = lane % CH, kv = lane / CH;  // lanes 0..CH-1: K, CH..2CH-1: V
+      const bool bad = (bad_mask >> st) & 1u;
+      // Where the tile lies. A shared tile counts for every member's columns,
+      // an own tile for its member's only.
+      int tok0, valid, mem, len;  // mem = -1: shared
+      bool use0, use1, has_new;
+      if (one_seq) {
+        tok0 = (tile0 + tile_idx) * TILE;
+        len = L0;
+        valid = min(TILE, L0 - tok0);
+        mem = 0;
+        use0 = col0_live;
+        use1 = col1_live;
+        has_new = j == j_new;
+      } else {
+        const TileLoc loc = locate_tile(view, tile0 + tile_idx, lane);
+        tok0 = loc.tok0;
+        len = loc.len;
+        mem = loc.m;
+        valid = mem < 0 ? TILE : min(TILE, len - tok0);
+        use0 = mem < 0 ? col0_live : mc0 == mem;
+        use1 = mem < 0 ? col1_live : mc1 == mem;
+        has_new = a.k_new != nullptr && mem >= 0 && len - 1 < tok0 + TILE;
+      }
+
+      if (has_new && !bad) {
+        // Fused append: this tile holds token L-1 of member mem. Its K and V
+        // rows come from the new rows (whatever the pool slot held), and the
+        // same rows are written to the pool slot: that is the cache-append.
+        const int r = len - 1 - tok0;
+        const int e = e_ch, kv = kv_ch;
         if (lane < 2 * CH) {
-          const uint4 v = lds128(stage + kv * D * 2 + e * 16);
+          uint4 v;
+          if constexpr (Shape::STAGED_NEW)
+            v = lds128(smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES + Shape::QROWS_BYTES +
+                       kv * D * 2 + e * 16);
+          else
+            v = newest;
           const uint32_t tile_base = kv ? vs : ks;
           sts128(tile_base + (e >> 3) * HALF_BYTES + r * 128 + (((e & 7) ^ (r & 7)) << 4), v);
-          const int tok = t_begin + new_tok;
+          const int tok = len - 1;
           const int idx = U8 ? tile_idx * 2 + (r >> 3) : tile_idx;
-          const int blk = idx < DESC_IDS ? desc[slot].ids[idx]
-                                         : a.block_tables[(size_t)s * a.max_blocks + tok / B];
+          const int blk = idx < DESC_IDS
+                              ? desc[slot].ids[idx]
+                              : a.block_tables[(size_t)(s + mem) * a.max_blocks + tok / B];
           T *pool = static_cast<T *>(const_cast<void *>(kv ? a.v_pool : a.k_pool));
           *reinterpret_cast<uint4 *>(pool + (((size_t)blk * Hkv + h) * B + tok % B) * D + e * 8) = v;
         }
@@ -921,10 +1304,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       // ---- online softmax (heads 2c, 2c+1; tokens g, g+8) ----
       const bool ok0 = !bad && g < valid;
       const bool ok1 = !bad && g + 8 < valid;
-      const float x0 = ok0 ? (sa[0] + sb[0]) * sl2 : -INFINITY;
-      const float x1 = ok0 ? (sa[1] + sb[1]) * sl2 : -INFINITY;
-      const float x2 = ok1 ? (sa[2] + sb[2]) * sl2 : -INFINITY;
-      const float x3 = ok1 ? (sa[3] + sb[3]) * sl2 : -INFINITY;
+      const float x0 = ok0 && use0 ? (sa[0] + sb[0]) * sl2 : -INFINITY;
+      const float x1 = ok0 && use1 ? (sa[1] + sb[1]) * sl2 : -INFINITY;
+      const float x2 = ok1 && use0 ? (sa[2] + sb[2]) * sl2 : -INFINITY;
+      const float x3 = ok1 && use1 ? (sa[3] + sb[3]) * sl2 : -INFINITY;
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -986,7 +1369,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       __syncwarp();  // every lane is done with this stage before it is refilled
       ++done;
-      pump(false);
+      newest = newest_next;
+      if (Shape::RING_COMBINE && j + 1 == nt_w)
+        last_st = st;  // it takes this warp's combine rows; refilled after the next vote
+      else
+        pump(false);
     }
 
     // Full per-warp sums: add the 8 lanes that share a head pair.
@@ -997,41 +1384,69 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
 
     // ---- combine the consumer warps ----
-    // 1) each warp stores its unnormalised rows and (max, sum) per head
+    // 1) each warp stores its unnormalised rows and (max, sum) per column:
+    //    into its own combine area, or (RING_COMBINE) into the stage of its
+    //    last tile, where a warp without tiles stores nothing
+    float *cw = nullptr;
+    if constexpr (Shape::RING_COMBINE) {
+      if (last_st >= 0)
+        cw = reinterpret_cast<float *>(sm + (size_t)(warp * NSTAGE + last_st) *
+                                                Shape::STAGE_BYTES);
+    } else {
+      cw = reinterpret_cast<float *>(sm + Shape::COMBINE_OFF) + warp * Shape::CW_FLOATS;
+    }
+    if (cw != nullptr) {
 #pragma unroll
-    for (int mt = 0; mt < D / 16; ++mt) {
-      if (2 * c < NH) {
-        cw_me[(2 * c) * AS + 16 * mt + g] = acc[mt][0];
-        cw_me[(2 * c) * AS + 16 * mt + g + 8] = acc[mt][2];
+      for (int mt = 0; mt < D / 16; ++mt) {
+        if (2 * c < NH) {
+          cw[(2 * c) * AS + 16 * mt + g] = acc[mt][0];
+          cw[(2 * c) * AS + 16 * mt + g + 8] = acc[mt][2];
+        }
+        if (2 * c + 1 < NH) {
+          cw[(2 * c + 1) * AS + 16 * mt + g] = acc[mt][1];
+          cw[(2 * c + 1) * AS + 16 * mt + g + 8] = acc[mt][3];
+        }
       }
-      if (2 * c + 1 < NH) {
-        cw_me[(2 * c + 1) * AS + 16 * mt + g] = acc[mt][1];
-        cw_me[(2 * c + 1) * AS + 16 * mt + g + 8] = acc[mt][3];
+      if (g == 0) {
+        if (2 * c < NH) {
+          cw[NH * AS + 2 * c] = m0;
+          cw[NH * AS + NH + 2 * c] = l0;
+        }
+        if (2 * c + 1 < NH) {
+          cw[NH * AS + 2 * c + 1] = m1;
+          cw[NH * AS + NH + 2 * c + 1] = l1;
+        }
       }
+      if constexpr (Shape::RING_COMBINE)
+        fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
     }
-    if (g == 0) {
-      if (2 * c < NH) {
-        cw_me[NH * AS + 2 * c] = m0;
-        cw_me[NH * AS + NH + 2 * c] = l0;
-      }
-      if (2 * c + 1 < NH) {
-        cw_me[NH * AS + 2 * c + 1] = m1;
-        cw_me[NH * AS + NH + 2 * c + 1] = l1;
-      }
-    }
+    if (lane == 0) comb_stage[warp] = last_st;
     consumers_sync();
-    // 2) per head: warp weights 2^(m_w - M) / sum, and the log2-sum-exp
-    if (threadIdx.x < G) {
+    const float *area[NCW];  // each warp's combine rows, or null
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+      if constexpr (Shape::RING_COMBINE) {
+        const int st = comb_stage[w];
+        area[w] = st < 0 ? nullptr
+                         : reinterpret_cast<const float *>(
+                               sm + (size_t)(w * NSTAGE + st) * Shape::STAGE_BYTES);
+      } else {
+        area[w] = reinterpret_cast<const float *>(sm + Shape::COMBINE_OFF) + w * Shape::CW_FLOATS;
+      }
+    }
+    // 2) per column: warp weights 2^(m_w - M) / sum, and the log2-sum-exp
+    if (threadIdx.x < ncol) {
       const int n = threadIdx.x;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, comb[w * Shape::CW_FLOATS + NH * AS + n]);
+      for (int w = 0; w < NCW; ++w)
+        if (area[w]) M = fmaxf(M, area[w][NH * AS + n]);
       float f[NCW], den = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
-        const float mw = comb[w * Shape::CW_FLOATS + NH * AS + n];
+        const float mw = area[w] ? area[w][NH * AS + n] : -INFINITY;
         f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-        den += f[w] * comb[w * Shape::CW_FLOATS + NH * AS + NH + n];
+        if (area[w]) den += f[w] * area[w][NH * AS + NH + n];
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
@@ -1041,14 +1456,15 @@ __global__ void __launch_bounds__(THREADS, 2)
     consumers_sync();
     // 3) outputs
     const bool single = nparts <= 1;
-    for (int idx = threadIdx.x; idx < G * D; idx += NCW * 32) {
+    for (int idx = threadIdx.x; idx < ncol * D; idx += NCW * 32) {
       const int n = idx / D;
       const int dd = idx - n * D;
       float o = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w)
-        o += scales[n * NCW + w] * comb[w * Shape::CW_FLOATS + n * AS + dd];
-      const size_t row = (size_t)s * Hq + h * G + n;
+        if (area[w]) o += scales[n * NCW + w] * area[w][n * AS + dd];
+      const int mem = n / G;  // row n is query head h*G + n%G of member mem
+      const size_t row = (size_t)(s + mem) * Hq + h * G + (n - mem * G);
       if (single) {
         out[row * D + dd] = from_float<T>(o);
       } else {
@@ -1097,6 +1513,11 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   if (grid < 1) grid = 1;
   DecodeArgs b = a;
   b.grid = (int)grid;
+  // With 8 columns, rows left over by one sequence's G query heads are filled
+  // with the heads of further sequences that share a prefix with it (up to
+  // 8 / G of them); with 4 columns an item attends one sequence.
+  const int groups_of = NH / (a.num_heads / a.num_kv_heads);
+  b.max_group = Shape::STAGED_NEW ? 1 : max(1, min(MAX_MEMBERS, groups_of));
 
   // Both launches are programmatic dependents of what precedes them in the
   // stream. The plan may start while a previous decode call finishes (it
@@ -1128,12 +1549,16 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
 template <typename T, bool U8>
 cudaError_t launch_tc_t(const DecodeArgs &a, const CUtensorMap &tmK, const CUtensorMap &tmV,
                         cudaStream_t stream) {
+  // 4 score columns for 3 or 4 query heads per KV head (one sequence per
+  // item). Otherwise 8: the G heads of one sequence, or with G = 1, 2 the
+  // heads of up to 8 / G sequences that share a prefix.
   const int G = a.num_heads / a.num_kv_heads;
+  const bool four = G == 3 || G == 4;
   if (a.head_dim == 64)
-    return G <= 4 ? launch_tc<T, 64, 4, U8>(a, tmK, tmV, stream)
-                  : launch_tc<T, 64, 8, U8>(a, tmK, tmV, stream);
-  return G <= 4 ? launch_tc<T, 128, 4, U8>(a, tmK, tmV, stream)
-                : launch_tc<T, 128, 8, U8>(a, tmK, tmV, stream);
+    return four ? launch_tc<T, 64, 4, U8>(a, tmK, tmV, stream)
+                : launch_tc<T, 64, 8, U8>(a, tmK, tmV, stream);
+  return four ? launch_tc<T, 128, 4, U8>(a, tmK, tmV, stream)
+              : launch_tc<T, 128, 8, U8>(a, tmK, tmV, stream);
 }
 
 }  // namespace

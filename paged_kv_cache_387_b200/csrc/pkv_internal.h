@@ -34,7 +34,8 @@ struct DecodeArgs {
   const void *k_new;
   const void *v_new;
   // Work list of the persistent decode kernel (written by the plan kernel):
-  uint2 *work;         // [<= S*max_parts] {seq << 16 | partition, context length}, fulls first
+  uint2 *work;         // [<= S*max_parts] {seq << 16 | partition, context length, or
+                       //  1 << 31 | the leader's grp word for a group}
   int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries
   // Partition merging (split contexts). Partitions are merged in chunks of
   // MERGE_CHUNK; a context with more than one chunk is merged in two levels.
@@ -44,19 +45,25 @@ struct DecodeArgs {
   float *ws2_lse;      // [S][Hq][max_chunks] chunk log2-sum-exp, or null
   int max_chunks;      // ceil(max_parts / MERGE_CHUNK)
   int grid;            // CTAs of the decode grid (each takes item blockIdx.x first)
+  // Shared-prefix groups (written by the plan kernel, read back by it):
+  int max_group;       // most sequences one work item may attend together (1 = no groups)
+  int32_t *grp;        // [S] 0: own entry; -1: member of an earlier leader's group;
+                       //     > 0: leader, (members - 1) << 27 | shared 16-token tiles
+  int32_t *grp_tiles;  // [S] a leader's group tiles: shared + every member's own
   int unit8;           // 1 when block_size % 16 == 8: a 16-token tile is two 8-token units
                        // that may sit in different blocks
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
 
-// Decode workspace, in order: scheduling words (256 B), the work list, then
+// Decode workspace, in order: scheduling words (256 B), the work list, the
+// per-sequence group words (two int32 per sequence), then
 // (only when a context can span several partitions) the merge counters, the
 // partition outputs with their log2-sum-exp values, and (only when a context
 // can span several merge chunks) the chunk results. Each region is 256-byte
 // aligned.
 struct WorkspaceLayout {
-  size_t sched_off, work_off, cnt_off, cnt2_off, o_off, lse_off, o2_off, lse2_off, total;
+  size_t sched_off, work_off, grp_off, cnt_off, cnt2_off, o_off, lse_off, o2_off, lse2_off, total;
 };
 WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long long max_parts);
 

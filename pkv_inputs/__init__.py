@@ -25,10 +25,12 @@ from .workloads import (  # noqa: F401
     WORKLOADS,
     make_case,
     make_random_case,
+    make_sharing_case,
     make_shared_prefix_case,
     nan_fill_value,
 )
 from .accounting import (  # noqa: F401
     decode_algorithmic_bytes,
     kv_bytes_per_token,
+    unique_kv_bytes,
 )

@@ -35,3 +35,24 @@ def decode_algorithmic_bytes(context_lens: Iterable[int], num_heads: int,
         total += 2 * num_heads * head_dim * elem_bytes
         total += 4 * nb + 4
     return total
+
+
+def unique_kv_bytes(block_tables, context_lens, block_size: int, num_kv_heads: int,
+                    head_dim: int, elem_bytes: int) -> int:
+    """K and V bytes of the distinct physical blocks a decode step reads.
+
+    Sequences that share a block (forked samples, beams, cached prefixes) read
+    the same memory; counted once, with the most slots any of them reads from
+    it. This is the traffic a reader that fetches each shared block once must
+    move, the bound for the sharing workloads; the per-sequence sum of
+    decode_algorithmic_bytes counts a shared block once per reader.
+    """
+    best = {}
+    for row, L in zip(block_tables, context_lens):
+        L = int(L)
+        for j in range(-(-L // block_size)):
+            b = int(row[j])
+            n = min(block_size, L - j * block_size)
+            if n > best.get(b, 0):
+                best[b] = n
+    return sum(best.values()) * 2 * num_kv_heads * head_dim * elem_bytes

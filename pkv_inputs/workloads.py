@@ -215,6 +215,86 @@ def make_random_case(name: str, num_heads: int, num_kv_heads: int, head_dim: int
               "tokens": ntok, "poison": poison})
 
 
+def make_sharing_case(name: str, num_heads: int, num_kv_heads: int, head_dim: int,
+                      block_size: int, groups, dtype: torch.dtype, seed: int, device="cpu",
+                      with_append: bool = False, partition_size: int = DEFAULT_PARTITION,
+                      spare_blocks: int = 3) -> DecodeCase:
+    """A decode step over groups of sequences that share a prompt's blocks.
+
+    ``groups`` lists ``(prompt_len, own_lens)``: the group's sequences (adjacent
+    in the batch) all start with the same ``prompt_len`` tokens, then member
+    ``i`` has ``own_lens[i]`` tokens of its own. The prompt's full blocks are
+    shared (one physical block, referenced by every member's table, as after
+    forking: page "PagedAttention Analysis", section 4). A partly filled last
+    prompt block is copied into every member's own first block, as
+    copy-on-write leaves it. Placement is a seeded shuffle of the pool; unused
+    slots are NaN. With ``with_append`` each sequence's newest token is
+    returned as ``k_new``/``v_new`` with its slot (it must be one of the
+    member's own tokens).
+    """
+    B = block_size
+    rng = np.random.default_rng(seed)
+    gen = _generator(seed, device)
+    lens, shared_blocks, own_blocks = [], [], []
+    for prompt_len, own in groups:
+        nf = prompt_len // B
+        shared_blocks.append(nf)
+        for o in own:
+            L = prompt_len + int(o)
+            if with_append and (o < 1):
+                raise ValueError("the appended token must be a member's own token")
+            lens.append(L)
+            own_blocks.append(-(-L // B) - nf)
+    P = sum(shared_blocks) + sum(own_blocks) + spare_blocks
+    order = rng.permutation(P).tolist()
+    S = len(lens)
+    bt = np.full((S, max([1] + [-(-L // B) for L in lens])), -1, dtype=np.int32)
+    fill = float("nan")
+    k_pool = torch.full((P, num_kv_heads, B, head_dim), fill, dtype=dtype, device=device)
+    v_pool = torch.full_like(k_pool, fill)
+    q = _randn((S, num_heads, head_dim), gen, dtype, device)
+    k_new_rows, v_new_rows, slots = [], [], []
+    s = 0
+    for (prompt_len, own), nf in zip(groups, shared_blocks):
+        pk = _randn((prompt_len, num_kv_heads, head_dim), gen, dtype, device)
+        pv = _randn((prompt_len, num_kv_heads, head_dim), gen, dtype, device)
+        shared = [order.pop() for _ in range(nf)]
+        for o in own:
+            L = prompt_len + int(o)
+            nb = -(-L // B)
+            table = shared + [order.pop() for _ in range(nb - nf)]
+            bt[s, :nb] = table
+            ok = _randn((int(o), num_kv_heads, head_dim), gen, dtype, device)
+            ov = _randn((int(o), num_kv_heads, head_dim), gen, dtype, device)
+            kt = torch.cat([pk, ok])
+            vt = torch.cat([pv, ov])
+            t = np.arange(L)
+            keep = t < L - 1 if with_append else np.ones(L, dtype=bool)
+            ph = torch.as_tensor(np.asarray(table)[t[keep] // B], device=device)
+            sl = torch.as_tensor(t[keep] % B, device=device)
+            k_pool[ph, :, sl, :] = kt[torch.as_tensor(keep, device=device)]
+            v_pool[ph, :, sl, :] = vt[torch.as_tensor(keep, device=device)]
+            if with_append:
+                k_new_rows.append(kt[L - 1])
+                v_new_rows.append(vt[L - 1])
+                slots.append(table[(L - 1) // B] * B + (L - 1) % B)
+            s += 1
+    k_new = v_new = slot_mapping = None
+    if with_append:
+        k_new = torch.stack(k_new_rows).contiguous()
+        v_new = torch.stack(v_new_rows).contiguous()
+        slot_mapping = torch.as_tensor(np.asarray(slots, np.int64), device=device)
+    return DecodeCase(
+        name=name, q=q, k_pool=k_pool, v_pool=v_pool,
+        block_tables=torch.as_tensor(bt, dtype=torch.int32, device=device),
+        context_lens=torch.as_tensor(np.asarray(lens, np.int32), device=device),
+        num_heads=num_heads, num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=B,
+        scale=1.0 / math.sqrt(head_dim), partition_size=partition_size, k_new=k_new,
+        v_new=v_new, slot_mapping=slot_mapping,
+        meta={"seed": seed, "pool_blocks": P, "groups": [(int(pl), [int(o) for o in ow])
+                                                         for pl, ow in groups]})
+
+
 # ---------------------------------------------------------------------------
 # The five workloads
 # ---------------------------------------------------------------------------

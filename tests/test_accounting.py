@@ -33,3 +33,30 @@ def test_batch256_workload_bytes_are_the_recorded_ones():
     assert len(lens) == 256 and sum(lens) == 222307
     assert min(lens) >= 1 and max(lens) <= 4096
     assert decode_algorithmic_bytes(lens, 32, 8, 128, 16, 2) == 914820836
+
+
+def test_unique_bytes_count_a_shared_block_once():
+    from pkv_inputs.accounting import unique_kv_bytes
+    per_tok = 2 * 2 * 64 * 2  # Hkv 2, d64, 16-bit, K and V
+    # two sequences share blocks 7 and 3 (32 tokens), then own blocks 5 and 9
+    bt = [[7, 3, 5], [7, 3, 9]]
+    assert unique_kv_bytes(bt, [40, 35], 16, 2, 64, 2) == (32 + 8 + 3) * per_tok
+    # a block shared with different fill levels counts its fullest reader
+    assert unique_kv_bytes([[4], [4]], [5, 11], 16, 2, 64, 2) == 11 * per_tok
+    # no sharing: the unique bytes are the per-sequence K/V bytes
+    lens = [1, 16, 17]
+    bt = [[0], [1], [2, 3]]
+    kv = sum(2 * L * 2 * 64 * 2 for L in lens)
+    assert unique_kv_bytes(bt, lens, 16, 2, 64, 2) == kv
+
+
+def test_shared_prefix_workload_unique_bytes():
+    """16 prompts of 1000 tokens: 62 full blocks shared by 6 samples, and each
+    sample's own 8 prompt tokens plus 64 decoded ones (fp16, 40 KV heads)."""
+    from pkv_inputs import make_shared_prefix_case
+    from pkv_inputs.accounting import unique_kv_bytes
+    sp = make_shared_prefix_case(num_heads=4, num_kv_heads=4, head_dim=16)
+    st = sp.steps[-1]
+    got = unique_kv_bytes(st["block_tables"].tolist(), st["context_lens"].tolist(), 16, 4, 16, 2)
+    per_tok = 2 * 4 * 16 * 2
+    assert got == (16 * 992 + 96 * 72) * per_tok

@@ -53,18 +53,38 @@ def test_status_strings(lib):
 
 def test_workspace_arithmetic(lib):
     f = lib.pkv_decode_workspace_bytes
-    # scheduling words (256 B) + work list (8 bytes per (seq, partition)),
-    # each region rounded up to 256 B
-    assert f(8, 32, 128, 512, 512) == 256 + 256   # one partition: no partials
-    assert f(8, 32, 128, 100, 0) == 256 + 256     # unsplit
-    # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16): chunk and
-    # final merge counters, fp32 partition outputs + lse, chunk results + lse
+    rnd = lambda x: -(-x // 256) * 256
+
+    def expected(S, Hq, D, L, P):
+        # partial-result rows per (sequence, query head): the partitions of the
+        # longest context, at least two (a shared-prefix group may split in two)
+        parts = 1 if P == 0 else -(-max(L, 1) // P)
+        rows = max(parts, 2)
+        chunks = -(-rows // 16)
+        total = (256                                 # scheduling words
+                 + rnd(S * rows * 8)                 # work list
+                 + rnd(2 * S * 4)                    # group words
+                 + rnd(S * Hq * chunks * 4)          # chunk merge counters
+                 + rnd(S * Hq * 4)                   # final merge counters
+                 + rnd(S * Hq * rows * D * 4)        # fp32 partition outputs
+                 + rnd(S * Hq * rows * 4))           # their log2-sum-exp
+        if chunks > 1:                               # chunk results
+            total += rnd(S * Hq * chunks * D * 4) + rnd(S * Hq * chunks * 4)
+        return total
+
+    # one partition or unsplit: two rows all the same
+    assert f(8, 32, 128, 512, 512) == 256 + 256 + 256 + 1024 + 1024 + 8 * 32 * 2 * 128 * 4 + 2048
+    assert f(8, 32, 128, 100, 0) == expected(8, 32, 128, 100, 0)
+    # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16)
     S, Hq, D, P, C = 8, 32, 128, 256, 16
-    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + S * Hq * C * 4 + S * Hq * 4
+    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + 256 + S * Hq * C * 4 + S * Hq * 4
                                         + S * Hq * P * D * 4 + S * Hq * P * 4
                                         + S * Hq * C * D * 4 + S * Hq * C * 4)
     # 33 tokens in 16-token partitions = 3 partitions, one merge chunk
-    assert f(1, 1, 64, 33, 16) == 256 + 256 + 256 + 256 + 3 * 64 * 4 + 256
+    assert f(1, 1, 64, 33, 16) == 256 + 256 + 256 + 256 + 256 + 3 * 64 * 4 + 256
+    for args in [(100, 8, 64, 100, 0), (3, 40, 128, 1064, 2048), (256, 32, 128, 4096, 2048),
+                 (5, 2, 64, 20000, 16)]:
+        assert f(*args) == expected(*args), args
     assert f(0, 32, 128, 512, 512) == 0
 
 
@@ -131,23 +151,41 @@ def test_append_and_copy_argument_checks(lib):
     assert cp(FAKE, FAKE, None, 0, 2, 128, 16, 10, 1, None, None) == pkv.PKV_OK
 
 
+@pytest.mark.gpu
 def test_binding_refuses_cpu_tensors(lib):
+    """A device `out` with q (or the pools) left on the host: the binding
+    refuses the host input before anything reaches the library."""
     import torch
     x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
     k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
     bt = torch.zeros(2, 1, dtype=torch.int32)
-    with pytest.raises(ValueError):
+    out = torch.empty(2, 8, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
+        pkv.paged_attn_decode(out, x, k.cuda(), k.cuda(), bt.cuda(), bt[:, 0].cuda(), 0.1, 16)
+    with pytest.raises(ValueError, match="k_pool must be a CUDA tensor"):
+        pkv.paged_attn_decode(out, x.cuda(), k, k, bt.cuda(), bt[:, 0].cuda(), 0.1, 16)
+
+
+def test_binding_refuses_host_q(lib):
+    """q on the host is refused before anything reaches the library (no GPU needed)."""
+    import torch
+    x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
+    bt = torch.zeros(2, 1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="q must be a CUDA tensor"):
         pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
 
 
+@pytest.mark.gpu
 def test_binding_refuses_unpinned_host_output(lib):
     """A host `out` is accepted only when it is page-locked."""
     import torch
-    x = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
-    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16)
-    bt = torch.zeros(2, 1, dtype=torch.int32)
+    x = torch.zeros(2, 8, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(4, 2, 16, 128, dtype=torch.bfloat16, device="cuda")
+    bt = torch.zeros(2, 1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="pinned"):
-        pkv.paged_attn_decode(x.clone(), x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
+        pkv.paged_attn_decode(out, x, k, k, bt, bt[:, 0].contiguous(), 0.1, 16)
 
 
 def test_wait_timeout_check_arguments(lib):

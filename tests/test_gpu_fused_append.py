@@ -148,3 +148,32 @@ def test_lengths_advanced_on_device_just_before_each_call(part):
         assert_close_to_oracle(out, ref, dt, f"device-advanced lengths, step {step}")
     assert torch.equal(kd.cpu().view(torch.int16), kc.view(torch.int16))
     assert torch.equal(vd.cpu().view(torch.int16), vc.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# the timed workloads at full size, every output, through the benchmarked call
+# ---------------------------------------------------------------------------
+
+def test_full_batch256_gqa_step_as_benchmarked():
+    """The batch-256 GQA step exactly as the benchmark times it: one
+    paged_attn_decode_append call with 2048-token partitions. All 256
+    sequences' outputs (every query head, every element) are compared with the
+    oracle's decode over the appended cache, and both pools with the oracle's
+    append, bit for bit (page "PagedAttention", newikis, section "Mathematical
+    formulation"; page "PagedAttention Analysis", section 3: the block-wise
+    walk equals ordinary attention)."""
+    c = make_case("llama8b_gqa_b256", device=DEV, with_append=True)
+    assert c.num_seqs == 256 and c.partition_size == 2048
+    fused_vs_oracle(c, c.partition_size, "batch-256 GQA, full batch, fused")
+
+
+def test_full_long_split_step_as_benchmarked():
+    """The long-context workload (8 sequences of 32768-131072 tokens, block 32)
+    at its 512-token partitions, through the fused call the benchmark times:
+    every output of all 8 sequences against the oracle, pools bit-exact. Each
+    context spans 64-256 partitions, so every one goes through the two-level
+    log-sum-exp merge."""
+    c = make_case("long_split_b8", device=DEV, with_append=True)
+    assert c.num_seqs == 8 and c.partition_size == 512
+    assert int(c.context_lens.min()) > 16 * 512  # more than one merge chunk each
+    fused_vs_oracle(c, c.partition_size, "long split, all 8 sequences, fused")

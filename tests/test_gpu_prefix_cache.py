@@ -2,8 +2,8 @@
 keyed by a hash of the whole prefix are shared through a global table. The
 cache's hits must be exactly the full blocks whose token prefix was seen
 before; the fused append + decode over the shared blocks must match the
-oracle; and the same requests laid out in private blocks must decode to the
-same bits."""
+oracle; and the same requests laid out in private blocks must decode to the same
+values."""
 
 import pytest
 import torch
@@ -69,4 +69,10 @@ def test_prefix_cache_sharing_decode(dt, B, Hq, Hkv, D):
                           partition_size=64, err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
+    # Requests that share cached blocks are attended together when a KV head
+    # serves at most 4 query heads (one work item reads each shared tile once),
+    # so the summation order differs from the private layout's: both must match
+    # the oracle. With larger groups both layouts run the same arithmetic.
+    assert_close_to_oracle(out2, ref, dt, "prefix cache, private blocks")
+    if Hq // Hkv > 4:
+        assert torch.equal(out2.view(torch.int16), out.view(torch.int16))
