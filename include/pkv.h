@@ -76,13 +76,11 @@ enum {
 /*
  * Bytes of device workspace paged_attn_decode needs for these sizes: a few
  * scheduling words, the work list (one 8-byte entry per possible
- * (sequence, partition) pair), two int32 per sequence for the shared-prefix
- * grouping, merge counters, and R fp32 output rows plus R fp32 log-sum-exp
- * values per (sequence, query head), where R is the partition count of a
- * max_context_len context, and at least 2 (the work of sequences that share
- * a prefix may be split in two even when no single context needs a split).
- * Always > 0 for num_seqs > 0. This function is pure arithmetic: it does not
- * touch the GPU.
+ * (sequence, partition) pair) and two int32 per sequence for the
+ * shared-prefix grouping, plus, when a context can span several
+ * partitions, merge counters and one fp32 output row and one fp32
+ * log-sum-exp per (sequence, query head, partition). Always > 0 for
+ * num_seqs > 0. This function is pure arithmetic: it does not touch the GPU.
  */
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_context_len, int partition_size);

@@ -22,15 +22,6 @@ long long parts_for(int max_context_len, int partition_size) {
   return (L + partition_size - 1) / partition_size;
 }
 
-// Partial-result rows per (sequence, query head) in the workspace: the
-// partitions of the longest context, and at least two, so that the work item
-// of a group of sequences that share a prefix can be split in two for balance
-// even when no single context needs splitting.
-long long part_rows_for(int max_context_len, int partition_size) {
-  const long long mp = parts_for(max_context_len, partition_size);
-  return mp < 2 ? 2 : mp;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -155,8 +146,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int
   if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || max_context_len < 0 ||
       partition_size < 0)
     return 0;
-  const long long rows = part_rows_for(max_context_len, partition_size);
-  return pkv::workspace_layout(num_seqs, num_heads, head_dim, rows).total;
+  const long long mp = parts_for(max_context_len, partition_size);
+  return pkv::workspace_layout(num_seqs, num_heads, head_dim, mp).total;
 }
 
 }  // extern "C"
@@ -198,8 +189,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
     if (rows > 0x7fffffffLL - 64) return PKV_EUNSUPPORTED;
   }
   const long long mp = parts_for(max_context_len, partition_size);
-  const long long prow = part_rows_for(max_context_len, partition_size);
-  if (prow > 65535) return PKV_EUNSUPPORTED;  // work-list entries pack the partition in 16 bits
+  if (mp > 65535) return PKV_EUNSUPPORTED;  // work-list entries pack the partition in 16 bits
   pkv::DecodeArgs a{};
   a.out = out;
   a.q = q;
@@ -216,7 +206,7 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
   a.max_context_len = max_context_len;
-  a.max_parts = (int)prow;
+  a.max_parts = (int)mp;
   if (partition_size > 0) {
     a.part_tokens = partition_size;
   } else {
@@ -226,15 +216,15 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
   }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.err = err;
-  const pkv::WorkspaceLayout wl = pkv::workspace_layout(num_seqs, num_heads, head_dim, prow);
+  const pkv::WorkspaceLayout wl = pkv::workspace_layout(num_seqs, num_heads, head_dim, mp);
   if (!workspace || workspace_bytes < wl.total || !aligned(workspace, 256)) return PKV_EINVAL;
   char *ws = static_cast<char *>(workspace);
   a.sched = reinterpret_cast<int32_t *>(ws + wl.sched_off);
   a.work = reinterpret_cast<uint2 *>(ws + wl.work_off);
   a.grp = reinterpret_cast<int32_t *>(ws + wl.grp_off);
   a.grp_tiles = a.grp + num_seqs;
-  a.max_chunks = (int)((prow + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK);
-  {
+  a.max_chunks = (int)((mp + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK);
+  if (mp > 1) {
     a.merge_cnt = reinterpret_cast<int32_t *>(ws + wl.cnt_off);
     a.merge_cnt2 = reinterpret_cast<int32_t *>(ws + wl.cnt2_off);
     if (a.max_chunks > 1) {

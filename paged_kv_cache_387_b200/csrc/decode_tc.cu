@@ -69,6 +69,7 @@
 // CTA-wide stop flag, and the kernel winds down, first waiting (bounded) for
 // the copies it still has in flight.
 #include <climits>
+#include <type_traits>
 
 #include "pkv_device.cuh"
 #include "pkv_internal.h"
@@ -141,15 +142,20 @@ struct TcShape {
   // two stages only. With 4 columns the area fits beside three stages, and a
   // warp refills its last stage at once.
   static constexpr bool RING_COMBINE = NH >= 8;
+  // Shared-prefix groups (several sequences per item) only with 8 columns.
+  static constexpr bool GROUPS = NH >= 8;
   static_assert(!RING_COMBINE || CW_FLOATS * 4 <= STAGE_BYTES, "a stage holds the rows");
-  static constexpr int COMBINE_BYTES = RING_COMBINE ? 0 : NCW * CW_FLOATS * 4;
+  // With 8 columns, items of at most SMALL_COLS columns (one sequence with
+  // G <= 2) still combine in a small area of their own and hold no stage.
+  static constexpr int SMALL_COLS = 2;
+  static constexpr int SMALL_CW = SMALL_COLS * ACC_STRIDE + 2 * SMALL_COLS;
+  static constexpr int COMBINE_BYTES = NCW * (RING_COMBINE ? SMALL_CW : CW_FLOATS) * 4;
   // weights [NH][NCW], log2-sum-exp [NH], each warp's combine stage [NCW]
   static constexpr int SCALES_BYTES = (NH * (NCW + 1) + NCW) * 4;
-  // One sequence per item (4 columns): its newest K and V rows travel with
-  // its q rows; groups (8 columns) read them from k_new / v_new.
-  static constexpr bool STAGED_NEW = !RING_COMBINE;
+  // An item of one sequence gets its newest K and V rows (fused append)
+  // with its q rows; a group's members read theirs from k_new / v_new.
   static constexpr int QROWS_BYTES = NH * D * 2;  // the q rows of every member
-  static constexpr int QBUF_BYTES = QROWS_BYTES + (STAGED_NEW ? 2 * D * 2 : 0);
+  static constexpr int QBUF_BYTES = QROWS_BYTES + 2 * D * 2;
   static constexpr int FIXED = COMBINE_BYTES + ((SCALES_BYTES + 15) & ~15) +
                                NSLOT * QBUF_BYTES + NSLOT * (int)sizeof(ItemDesc) + 64 * 8 +
                                1024 + 64;
@@ -177,18 +183,13 @@ __device__ __forceinline__ uint32_t pack_pair(int s, int p) {
 }
 
 // Tiles per partition of an entry. One sequence uses the call's partition
-// length. A group of sequences that share a prefix (see plan_groups) spans its
-// shared tiles once plus every member's own tiles; it is cut into balanced
-// partitions of at most GROUP_PART_TILES tiles (or the call's length, if
-// shorter), as many as the workspace rows each member has (max_parts) allow,
-// so that a few large group items do not leave most CTAs idle at the end.
-constexpr int GROUP_PART_TILES = 64;
+// length. A group of sequences that share a prefix (see plan_group_round) spans its
+// shared tiles once plus every member's own tiles; it uses partitions long
+// enough that their number never exceeds max_parts, so each member's partial
+// results fit its workspace rows.
 __device__ __forceinline__ int group_part_tiles(const DecodeArgs &a, bool grouped, int tiles) {
   const int pt = a.part_tokens / TILE;
-  if (!grouped) return pt;
-  const int want = min(pt, GROUP_PART_TILES);
-  const int np = max(1, min(a.max_parts, (tiles + want - 1) / want));
-  return max(1, (tiles + np - 1) / np);
+  return grouped ? max(pt, (tiles + a.max_parts - 1) / a.max_parts) : pt;
 }
 
 // Inclusive prefix maximum over the plan block (one value per thread).
@@ -234,11 +235,15 @@ __device__ __forceinline__ int plan_block_max_scan(int v, int *wmax) {
 // The table comparison touches only candidate pairs (equal first entries) and
 // only the entries that both sequences' shared span covers, spread over all
 // threads of the block.
-// Returns whether any group formed (uniform over the block); when none did,
-// a.grp is not written and the caller treats every sequence as its own.
-template <typename EffLen, typename BlockScan>
-__device__ __noinline__ bool plan_groups(const DecodeArgs &a, EffLen eff_len,
-                                         BlockScan block_scan) {
+// One round of PLAN_THREADS sequences (thread tid holds sequence s = r0 + tid,
+// of clamped length L) that has at least one candidate pair (cand: s-1 and s
+// may share `cap` tiles and their first table entries agree). Sets this
+// thread's group word and, for a leader, the group's tiles, and stores both
+// in a.grp / a.grp_tiles for the plan's second pass.
+template <typename BlockScan>
+__device__ __noinline__ void plan_group_round(const DecodeArgs &a, int s, int L, int cap,
+                                              bool cand, BlockScan block_scan, int &word,
+                                              int &gtiles) {
   __shared__ int c_seq[PLAN_THREADS];     // candidate pairs (s-1, s): s
   __shared__ int c_off[PLAN_THREADS];     // first comparison index of each candidate
   __shared__ int c_mis[PLAN_THREADS];     // first differing block (or the blocks compared)
@@ -248,80 +253,74 @@ __device__ __noinline__ bool plan_groups(const DecodeArgs &a, EffLen eff_len,
   __shared__ int wmax[PLAN_THREADS / 32];
   const int tid = threadIdx.x;
   const int S = a.num_seqs, B = a.block_size;
-  const int newest = a.k_new != nullptr ? 1 : 0;
-  bool any = false;
-  for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
-    const int s = r0 + tid;
-    const int L = s < S ? eff_len(s) : 0;
-    int cap = 0;  // tiles the pair (s-1, s) could share
-    bool cand = false;
-    if (s < S && tid > 0) {
-      // (the first entries are loaded with the lengths; they count only if cap > 0)
-      const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
-      const int32_t b_this = bt[0], b_prev = (bt - a.max_blocks)[0];  // row s-1 precedes row s
-      cap = (min(L, eff_len(s - 1)) - newest) / TILE;
-      cand = cap > 0 && b_this == b_prev;
-    }
-    const int nblk = cand ? (cap * TILE + B - 1) / B : 0;  // blocks covering the span
-    int ncand, work;
-    const int ci = block_scan(cand ? 1 : 0, ncand);
-    if (ncand == 0) {  // (uniform) no pair of this round starts with the same block
-      if (any && s < S) a.grp[s] = 0;
-      continue;
-    }
-    if (!any) {  // the earlier rounds had no group: record them as single sequences
-      for (int i = tid; i < r0; i += PLAN_THREADS) a.grp[i] = 0;
-      any = true;
-    }
-    const int co = block_scan(cand ? nblk - 1 : 0, work);  // block 0 is already compared
-    if (cand) {
-      c_seq[ci] = s;
-      c_off[ci] = co;
-      c_mis[ci] = nblk;
-    }
-    g_cnt[tid] = 0;
-    g_sh[tid] = INT_MAX;
-    g_own[tid] = 0;
-    __syncthreads();
-    // every comparison of every candidate: f -> (candidate c, block j >= 1)
-    for (int f = tid; f < work; f += PLAN_THREADS) {
-      int lo = 0, hi = ncand - 1;  // the last candidate whose range starts at or before f
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (c_off[mid] <= f)
-          lo = mid;
-        else
-          hi = mid - 1;
-      }
-      const int j = f - c_off[lo] + 1;
-      if (j < *static_cast<volatile int *>(&c_mis[lo])) {  // skip past a known difference
-        const int32_t *bt = a.block_tables + (size_t)c_seq[lo] * a.max_blocks;
-        if (bt[j] != (bt - a.max_blocks)[j]) atomicMin(&c_mis[lo], j);
-      }
-    }
-    __syncthreads();
-    const int psh = cand ? min(c_mis[ci] * B / TILE, cap) : 0;
-    const bool linked = psh > 0;  // never for tid 0: runs do not cross rounds
-    const int run = plan_block_max_scan(linked ? -1 : tid, wmax);
-    const int lead = run + (tid - run) / a.max_group * a.max_group;
-    if (s < S) {
-      atomicAdd(&g_cnt[lead], 1);
-      if (tid != lead) atomicMin(&g_sh[lead], psh);
-    }
-    __syncthreads();
-    const int members = g_cnt[lead];
-    const int sh = members > 1 ? g_sh[lead] : 0;
-    if (s < S && members > 1) atomicAdd(&g_own[lead], (L - sh * TILE + TILE - 1) / TILE);
-    __syncthreads();
-    if (s < S) {
-      int word = 0;
-      if (members > 1) word = tid == lead ? ((members - 1) << 27) | sh : -1;
-      a.grp[s] = word;
-      if (word > 0) a.grp_tiles[s] = sh + g_own[lead];
-    }
-    __syncthreads();  // the shared arrays are rewritten by the next round
+  const int nblk = cand ? (cap * TILE + B - 1) / B : 0;  // blocks covering the span
+  int ncand, work;
+  const int ci = block_scan(cand ? 1 : 0, ncand);
+  const int co = block_scan(cand ? nblk - 1 : 0, work);  // block 0 is already compared
+  if (cand) {
+    c_seq[ci] = s;
+    c_off[ci] = co;
+    c_mis[ci] = nblk;
   }
-  return any;
+  g_cnt[tid] = 0;
+  g_sh[tid] = INT_MAX;
+  g_own[tid] = 0;
+  __syncthreads();
+  // every comparison of every candidate: f -> (candidate c, block j >= 1).
+  // A thread takes CMP_BATCH consecutive comparisons and issues all their
+  // table loads before it compares, so that their latencies overlap.
+  constexpr int CMP_BATCH = 32;
+  for (int f0 = tid * CMP_BATCH; f0 < work; f0 += PLAN_THREADS * CMP_BATCH) {
+    int lo = 0, hi = ncand - 1;  // the last candidate whose range starts at or before f0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (c_off[mid] <= f0)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    int c = lo;
+    int cc[CMP_BATCH], jj[CMP_BATCH], va[CMP_BATCH], vb[CMP_BATCH];
+#pragma unroll
+    for (int k = 0; k < CMP_BATCH; ++k) {
+      const int f = f0 + k;
+      while (c + 1 < ncand && c_off[c + 1] <= f) ++c;  // the candidate holding f
+      cc[k] = f < work ? c : -1;
+      jj[k] = f - c_off[c] + 1;
+      va[k] = vb[k] = 0;
+      if (f < work) {
+        const int32_t *bt = a.block_tables + (size_t)c_seq[c] * a.max_blocks;
+        va[k] = bt[jj[k]];
+        vb[k] = (bt - a.max_blocks)[jj[k]];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < CMP_BATCH; ++k)
+      if (cc[k] >= 0 && va[k] != vb[k]) atomicMin(&c_mis[cc[k]], jj[k]);
+  }
+  __syncthreads();
+  const int psh = cand ? min(c_mis[ci] * B / TILE, cap) : 0;
+  const bool linked = psh > 0;  // never for tid 0: runs do not cross rounds
+  const int run = plan_block_max_scan(linked ? -1 : tid, wmax);
+  const int lead = run + (tid - run) / a.max_group * a.max_group;
+  if (s < S) {
+    atomicAdd(&g_cnt[lead], 1);
+    if (tid != lead) atomicMin(&g_sh[lead], psh);
+  }
+  __syncthreads();
+  const int members = g_cnt[lead];
+  const int sh = members > 1 ? g_sh[lead] : 0;
+  if (s < S && members > 1) atomicAdd(&g_own[lead], (L - sh * TILE + TILE - 1) / TILE);
+  __syncthreads();
+  word = 0;
+  gtiles = 0;
+  if (s < S) {
+    if (members > 1) word = tid == lead ? ((members - 1) << 27) | sh : -1;
+    if (word > 0) gtiles = sh + g_own[lead];
+    a.grp[s] = word;
+    if (word > 0) a.grp_tiles[s] = gtiles;
+  }
+  __syncthreads();  // the shared arrays are rewritten by the next round
 }
 
 // Build the work list in two regions.
@@ -335,7 +334,7 @@ __device__ __noinline__ bool plan_groups(const DecodeArgs &a, EffLen eff_len,
 //     order. A sequence of length 0 is one (empty) entry, so that its output
 //     is still written.
 // An entry is one sequence, or, when a.max_group > 1, one group of adjacent
-// sequences that share their first blocks (plan_groups): the group's leader
+// sequences that share their first blocks (plan_group_round): the group's leader
 // carries it and the other members have no entry. Each entry carries the
 // sequence's clamped length, or the leader's group word. Sequences are taken
 // in rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t),
@@ -360,7 +359,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   uint2 *const list = a.work;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs;
-  bool grouping = a.max_group > 1;
+  const bool grouping = a.max_group > 1;
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
   if (tid == 0) bad_len = 0;
   __syncthreads();
@@ -399,12 +398,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
                          nullptr);
   };
 
-  if (grouping) grouping = plan_groups(a, eff_len, block_scan);
-
-  // Tiles and partitions of sequence s's entry (np = 0: no entry; a group
-  // member other than the leader). `word` is the entry's second field.
-  auto entry_shape = [&](int s, int L, int &np, int &tiles, uint32_t &word) {
-    const int g = grouping ? a.grp[s] : 0;
+  // Tiles and partitions of sequence s's entry from its group word g (np = 0:
+  // no entry, a group member other than the leader). `word` is the entry's
+  // second field.
+  auto entry_shape = [&](int L, int g, int gtiles, int &np, int &tiles, uint32_t &word) {
     word = (uint32_t)L;
     tiles = (L + TILE - 1) / TILE;
     if (g < 0) {
@@ -412,24 +409,60 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
       return;
     }
     if (g > 0) {
-      tiles = a.grp_tiles[s];
+      tiles = gtiles;
       word = 0x80000000u | (uint32_t)g;
     }
     const int ptg = group_part_tiles(a, g > 0, tiles);
     np = max(1, (tiles + ptg - 1) / ptg);  // an empty sequence still has its (empty) entry
   };
 
-  // pass 1: region-1 entry count and the size-class histogram of region 2
+  // pass 1: the shared-prefix groups of each round, the region-1 entry count
+  // and the size-class histogram of region 2. With groups possible, each
+  // thread loads its predecessor's length and both first table entries with
+  // its own length; a round where no pair of first entries agrees costs one
+  // more barrier.
+  const int newest = a.k_new != nullptr ? 1 : 0;
+  bool any_group = false;  // (uniform) a group formed: the words are in a.grp
   int nm = 0;
   for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
     const int s = r0 + tid;
+    int raw = 0, raw_prev = 0;
+    int32_t b_this = 0, b_prev = 0;
     if (s < S) {
-      const int raw = a.context_lens[s];
-      const int L = eff_len(s);
-      if (L < raw) bad_len = 1;
+      raw = a.context_lens[s];
+      if (grouping && tid > 0) {  // (runs do not cross rounds)
+        const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
+        raw_prev = a.context_lens[s - 1];
+        b_this = bt[0];
+        b_prev = (bt - a.max_blocks)[0];  // row s-1 precedes row s
+      }
+    }
+    const int L = s < S ? effective_len(raw, a.max_context_len, a.max_blocks, a.block_size,
+                                        nullptr)
+                        : 0;
+    if (s < S && L < raw) bad_len = 1;
+    int word = 0, gtiles = 0;
+    if (grouping) {
+      int cap = 0;  // tiles the pair (s-1, s) could share
+      if (s < S && tid > 0)
+        cap = (min(L, effective_len(raw_prev, a.max_context_len, a.max_blocks, a.block_size,
+                                    nullptr)) -
+               newest) / TILE;
+      const bool cand = cap > 0 && b_this == b_prev;
+      if (__syncthreads_or(cand)) {
+        if (!any_group) {  // the earlier rounds had no group: record them as single sequences
+          for (int i = tid; i < r0; i += PLAN_THREADS) a.grp[i] = 0;
+          any_group = true;
+        }
+        plan_group_round(a, s, L, cap, cand, block_scan, word, gtiles);
+      } else if (any_group && s < S) {
+        a.grp[s] = 0;
+      }
+    }
+    if (s < S) {
       int np, tiles;
-      uint32_t word;
-      entry_shape(s, L, np, tiles, word);
+      uint32_t w;
+      entry_shape(L, word, gtiles, np, tiles, w);
       if (np > 1)
         nm += np;
       else if (np == 1)
@@ -462,7 +495,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     uint32_t word = 0;
     if (s < S) {
       int n, tiles;
-      entry_shape(s, eff_len(s), n, tiles, word);
+      const int g = any_group ? a.grp[s] : 0;
+      entry_shape(eff_len(s), g, g > 0 ? a.grp_tiles[s] : 0, n, tiles, word);
       if (n > 1)
         np = n;
       else if (n == 1)
@@ -697,9 +731,11 @@ __device__ __forceinline__ ItemView item_view(const ItemDesc &d, int lane) {
   return v;
 }
 
-// Called by all lanes of a warp with the same gt.
+// Called by all lanes of a warp with the same gt. GROUPS: the item may attend
+// several sequences.
+template <bool GROUPS>
 __device__ __forceinline__ TileLoc locate_tile(const ItemView &v, int gt, int lane) {
-  if (v.members == 1) return TileLoc{0, gt * TILE, v.len0};  // one sequence: all its own
+  if (!GROUPS || v.members == 1) return TileLoc{0, gt * TILE, v.len0};  // one sequence
   if (gt < v.sh) return TileLoc{-1, gt * TILE, INT_MAX};
   // own[] is non-decreasing: the member is the number of later members that
   // start at or before gt (lanes past the members hold INT_MAX)
@@ -868,7 +904,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       // One sequence (its clamped length in the entry), or a shared-prefix
       // group led by s (its members' lengths are read here, clamped as the
       // plan clamped them).
-      const bool grouped = (wk.y >> 31) != 0;
+      const bool grouped = Shape::GROUPS && (wk.y >> 31) != 0;
       const int members =  // (the plan never forms more; the bounds keep every copy in place)
           grouped ? min((int)((wk.y >> 27) & 15u) + 1,
                         min(min(MAX_MEMBERS, max(1, NH / G)), a.num_seqs - s))
@@ -904,7 +940,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       // and the arrival that publishes the descriptor comes last.
       const uint32_t qbytes = n_tiles > 0 ? (uint32_t)(G * D * 2) : 0u;
       const uint32_t stage = smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES;
-      if constexpr (Shape::STAGED_NEW) {  // one sequence: lane 0 issues everything
+      if (!grouped) {  // one sequence: lane 0 issues everything
         const int last = own_n - 1;       // its last tile holds token L-1
         const uint32_t rbytes =
             a.k_new != nullptr && last >= tile0 && last < tile0 + n_tiles ? (uint32_t)(D * 2) : 0u;
@@ -1068,9 +1104,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       const int tile = warp + is_j * NCW;
       const ItemDesc &dd = desc[is_it % NSLOT];
-      const TileLoc loc = locate_tile(is_view, is_tile0 + tile, lane);
+      const TileLoc loc = locate_tile<Shape::GROUPS>(is_view, is_tile0 + tile, lane);
       const int tok0 = loc.tok0;
-      const size_t trow = (size_t)(is_s + max(loc.m, 0)) * a.max_blocks;  // its table row
+      const size_t trow =  // its table row
+          (size_t)(Shape::GROUPS ? is_s + max(loc.m, 0) : is_s) * a.max_blocks;
       const int st = issued % NSTAGE;
       // Pool row of each unit of the tile. total_rows is wholly out of
       // bounds, and TMA fills zeros there. It is used for an invalid block id,
@@ -1153,7 +1190,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int s = dref.s, p = dref.p, h = dref.h, n_tiles = dref.n_tiles;
     const int nparts = dref.nparts;
     const int members = dref.members, tile0 = dref.tile0;
-    const bool one_seq = members == 1;
+    const bool one_seq = !Shape::GROUPS || members == 1;
     const int ncol = members * G;  // head rows attended: G per member
     // this lane's two columns (query heads 2c, 2c+1 of the rows) belong to these members
     const bool col0_live = mc0 < members, col1_live = mc1 < members;
@@ -1179,7 +1216,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     float m0 = -INFINITY, m1 = -INFINITY;  // reference max of heads 2c, 2c+1 (base-2 units)
     float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
     bool aborted = false;
-    int last_st = -1;  // with RING_COMBINE: the stage of this warp's last tile of the item
+    // Combine rows: `rows` columns per warp, in the combine area or (held) in
+    // the ring stage of the warp's last tile of the item (last_st).
+    const bool held = Shape::RING_COMBINE && ncol > Shape::SMALL_COLS;
+    const int rows = held || !Shape::RING_COMBINE ? NH : Shape::SMALL_COLS;
+    int last_st = -1;
 
     const ItemView view = item_view(dref, lane);
     const int L0 = view.len0;  // one sequence: its length
@@ -1189,32 +1230,29 @@ __global__ void __launch_bounds__(THREADS, 2)
       const int idx = (L0 - 1) / TILE - tile0;
       if (idx >= 0 && idx < n_tiles && idx % NCW == warp) j_new = idx / NCW;
     }
-    // Fused append, 8 columns: the K (lanes < CH) or V (lanes CH..2CH-1) row
+    // Fused append, a group: the K (lanes < CH) or V (lanes CH..2CH-1) row
     // chunk of the newest token of the member whose last tile is this warp's
     // j-th tile, read from k_new / v_new one tile before it is used.
     auto fetch_newest = [&](int j) {
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if constexpr (!Shape::STAGED_NEW) {
-        if (a.k_new == nullptr || j >= nt_w) return v;  // (uniform)
-        int m = 0;
-        if (one_seq) {
-          if (j != j_new) return v;
-        } else {
-          const TileLoc l = locate_tile(view, tile0 + warp + j * NCW, lane);
-          if (l.m < 0 || l.len - 1 >= l.tok0 + TILE) return v;
-          m = l.m;
-        }
-        if (lane >= 2 * CH) return v;
+      if constexpr (Shape::GROUPS) {
+        // (one sequence: its rows were staged with its q rows)
+        if (a.k_new == nullptr || one_seq || j >= nt_w) return v;  // (uniform)
+        const TileLoc l = locate_tile<Shape::GROUPS>(view, tile0 + warp + j * NCW, lane);
+        if (l.m < 0 || l.len - 1 >= l.tok0 + TILE || lane >= 2 * CH) return v;
         const T *src = static_cast<const T *>(kv_ch ? a.v_new : a.k_new) +
-                       ((size_t)(s + m) * Hkv + h) * D + e_ch * 8;
+                       ((size_t)(s + l.m) * Hkv + h) * D + e_ch * 8;
         v = __ldg(reinterpret_cast<const uint4 *>(src));
       }
       return v;
     };
-    uint4 newest = fetch_newest(0);
-
+    // The tile loop, compiled once for one sequence per item (GRP false: plain
+    // tile arithmetic) and once for a group (shared and own tiles).
+    auto run_tiles = [&](auto grp_tag) {
+    constexpr bool GRP = decltype(grp_tag)::value;
+    uint4 newest = GRP ? fetch_newest(0) : make_uint4(0u, 0u, 0u, 0u);
     for (int j = 0; j < nt_w; ++j) {
-      const uint4 newest_next = fetch_newest(j + 1);
+      const uint4 newest_next = GRP ? fetch_newest(j + 1) : make_uint4(0u, 0u, 0u, 0u);
       if (issued == done) pump(true);
       const int st = done % NSTAGE;
       if (issued == done ||
@@ -1231,7 +1269,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       // an own tile for its member's only.
       int tok0, valid, mem, len;  // mem = -1: shared
       bool use0, use1, has_new;
-      if (one_seq) {
+      if constexpr (!GRP) {
         tok0 = (tile0 + tile_idx) * TILE;
         len = L0;
         valid = min(TILE, L0 - tok0);
@@ -1240,7 +1278,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         use1 = col1_live;
         has_new = j == j_new;
       } else {
-        const TileLoc loc = locate_tile(view, tile0 + tile_idx, lane);
+        const TileLoc loc = locate_tile<Shape::GROUPS>(view, tile0 + tile_idx, lane);
         tok0 = loc.tok0;
         len = loc.len;
         mem = loc.m;
@@ -1258,7 +1296,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int e = e_ch, kv = kv_ch;
         if (lane < 2 * CH) {
           uint4 v;
-          if constexpr (Shape::STAGED_NEW)
+          if constexpr (!GRP)
             v = lds128(smem0 + Shape::QBUF_OFF + slot * Shape::QBUF_BYTES + Shape::QROWS_BYTES +
                        kv * D * 2 + e * 16);
           else
@@ -1350,7 +1388,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint32_t pb0 = movmatrix_trans(w01);  // tokens 0..7
       const uint32_t pb1 = movmatrix_trans(w23);  // tokens 8..15
       constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
-      uint32_t pl0 = 0, pl1 = 0;
+      [[maybe_unused]] uint32_t pl0 = 0, pl1 = 0;
       if constexpr (kSplitP) {
         pl0 = movmatrix_trans(pack2<T>(p0 - lo_half_to_float<T>(w01), p1 - hi_half_to_float<T>(w01)));
         pl1 = movmatrix_trans(pack2<T>(p2 - lo_half_to_float<T>(w23), p3 - hi_half_to_float<T>(w23)));
@@ -1370,11 +1408,16 @@ __global__ void __launch_bounds__(THREADS, 2)
       __syncwarp();  // every lane is done with this stage before it is refilled
       ++done;
       newest = newest_next;
-      if (Shape::RING_COMBINE && j + 1 == nt_w)
+      if (held && j + 1 == nt_w)
         last_st = st;  // it takes this warp's combine rows; refilled after the next vote
       else
         pump(false);
     }
+    };
+    if (Shape::GROUPS && !one_seq)
+      run_tiles(std::true_type{});
+    else
+      run_tiles(std::false_type{});
 
     // Full per-warp sums: add the 8 lanes that share a head pair.
 #pragma unroll
@@ -1385,53 +1428,54 @@ __global__ void __launch_bounds__(THREADS, 2)
 
     // ---- combine the consumer warps ----
     // 1) each warp stores its unnormalised rows and (max, sum) per column:
-    //    into its own combine area, or (RING_COMBINE) into the stage of its
-    //    last tile, where a warp without tiles stores nothing
+    //    into its own combine area, or (held) into the stage of its last
+    //    tile, where a warp without tiles stores nothing
+    const int cw_floats = rows * AS + 2 * rows;
+    float *const own_area = reinterpret_cast<float *>(sm + Shape::COMBINE_OFF);
     float *cw = nullptr;
-    if constexpr (Shape::RING_COMBINE) {
+    if (held) {
       if (last_st >= 0)
         cw = reinterpret_cast<float *>(sm + (size_t)(warp * NSTAGE + last_st) *
                                                 Shape::STAGE_BYTES);
     } else {
-      cw = reinterpret_cast<float *>(sm + Shape::COMBINE_OFF) + warp * Shape::CW_FLOATS;
+      cw = own_area + warp * cw_floats;
     }
     if (cw != nullptr) {
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) {
-        if (2 * c < NH) {
+        if (2 * c < rows) {
           cw[(2 * c) * AS + 16 * mt + g] = acc[mt][0];
           cw[(2 * c) * AS + 16 * mt + g + 8] = acc[mt][2];
         }
-        if (2 * c + 1 < NH) {
+        if (2 * c + 1 < rows) {
           cw[(2 * c + 1) * AS + 16 * mt + g] = acc[mt][1];
           cw[(2 * c + 1) * AS + 16 * mt + g + 8] = acc[mt][3];
         }
       }
       if (g == 0) {
-        if (2 * c < NH) {
-          cw[NH * AS + 2 * c] = m0;
-          cw[NH * AS + NH + 2 * c] = l0;
+        if (2 * c < rows) {
+          cw[rows * AS + 2 * c] = m0;
+          cw[rows * AS + rows + 2 * c] = l0;
         }
-        if (2 * c + 1 < NH) {
-          cw[NH * AS + 2 * c + 1] = m1;
-          cw[NH * AS + NH + 2 * c + 1] = l1;
+        if (2 * c + 1 < rows) {
+          cw[rows * AS + 2 * c + 1] = m1;
+          cw[rows * AS + rows + 2 * c + 1] = l1;
         }
       }
-      if constexpr (Shape::RING_COMBINE)
-        fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
+      if (held) fence_proxy_async_smem();  // these writes precede the stage's next TMA fill
     }
-    if (lane == 0) comb_stage[warp] = last_st;
+    if (held && lane == 0) comb_stage[warp] = last_st;
     consumers_sync();
     const float *area[NCW];  // each warp's combine rows, or null
 #pragma unroll
     for (int w = 0; w < NCW; ++w) {
-      if constexpr (Shape::RING_COMBINE) {
+      if (held) {
         const int st = comb_stage[w];
         area[w] = st < 0 ? nullptr
                          : reinterpret_cast<const float *>(
                                sm + (size_t)(w * NSTAGE + st) * Shape::STAGE_BYTES);
       } else {
-        area[w] = reinterpret_cast<const float *>(sm + Shape::COMBINE_OFF) + w * Shape::CW_FLOATS;
+        area[w] = own_area + w * cw_floats;
       }
     }
     // 2) per column: warp weights 2^(m_w - M) / sum, and the log2-sum-exp
@@ -1440,13 +1484,13 @@ __global__ void __launch_bounds__(THREADS, 2)
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NCW; ++w)
-        if (area[w]) M = fmaxf(M, area[w][NH * AS + n]);
+        if (area[w]) M = fmaxf(M, area[w][rows * AS + n]);
       float f[NCW], den = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) {
-        const float mw = area[w] ? area[w][NH * AS + n] : -INFINITY;
+        const float mw = area[w] ? area[w][rows * AS + n] : -INFINITY;
         f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
-        if (area[w]) den += f[w] * area[w][NH * AS + NH + n];
+        if (area[w]) den += f[w] * area[w][rows * AS + rows + n];
       }
       const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
@@ -1517,7 +1561,7 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   // with the heads of further sequences that share a prefix with it (up to
   // 8 / G of them); with 4 columns an item attends one sequence.
   const int groups_of = NH / (a.num_heads / a.num_kv_heads);
-  b.max_group = Shape::STAGED_NEW ? 1 : max(1, min(MAX_MEMBERS, groups_of));
+  b.max_group = Shape::GROUPS ? max(1, min(MAX_MEMBERS, groups_of)) : 1;
 
   // Both launches are programmatic dependents of what precedes them in the
   // stream. The plan may start while a previous decode call finishes (it

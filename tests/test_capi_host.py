@@ -56,26 +56,24 @@ def test_workspace_arithmetic(lib):
     rnd = lambda x: -(-x // 256) * 256
 
     def expected(S, Hq, D, L, P):
-        # partial-result rows per (sequence, query head): the partitions of the
-        # longest context, at least two (a shared-prefix group may split in two)
-        parts = 1 if P == 0 else -(-max(L, 1) // P)
-        rows = max(parts, 2)
-        chunks = -(-rows // 16)
-        total = (256                                 # scheduling words
-                 + rnd(S * rows * 8)                 # work list
-                 + rnd(2 * S * 4)                    # group words
-                 + rnd(S * Hq * chunks * 4)          # chunk merge counters
-                 + rnd(S * Hq * 4)                   # final merge counters
-                 + rnd(S * Hq * rows * D * 4)        # fp32 partition outputs
-                 + rnd(S * Hq * rows * 4))           # their log2-sum-exp
-        if chunks > 1:                               # chunk results
-            total += rnd(S * Hq * chunks * D * 4) + rnd(S * Hq * chunks * 4)
+        parts = 1 if P == 0 else -(-max(L, 1) // P)  # partitions of the longest context
+        total = 256 + rnd(S * parts * 8) + rnd(2 * S * 4)  # sched words, work list, group words
+        if parts > 1:
+            chunks = -(-parts // 16)
+            total += (rnd(S * Hq * chunks * 4) + rnd(S * Hq * 4)      # merge counters
+                      + rnd(S * Hq * parts * D * 4) + rnd(S * Hq * parts * 4))  # partials
+            if chunks > 1:                                             # chunk results
+                total += rnd(S * Hq * chunks * D * 4) + rnd(S * Hq * chunks * 4)
         return total
 
-    # one partition or unsplit: two rows all the same
-    assert f(8, 32, 128, 512, 512) == 256 + 256 + 256 + 1024 + 1024 + 8 * 32 * 2 * 128 * 4 + 2048
-    assert f(8, 32, 128, 100, 0) == expected(8, 32, 128, 100, 0)
-    # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16)
+    # scheduling words (256 B) + work list (8 bytes per (seq, partition)) +
+    # shared-prefix group words (two int32 per sequence), each region rounded
+    # up to 256 B
+    assert f(8, 32, 128, 512, 512) == 256 + 256 + 256   # one partition: no partials
+    assert f(8, 32, 128, 100, 0) == 256 + 256 + 256     # unsplit
+    assert f(100, 8, 64, 100, 0) == 256 + rnd(100 * 8) + rnd(100 * 8)
+    # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16): chunk and
+    # final merge counters, fp32 partition outputs + lse, chunk results + lse
     S, Hq, D, P, C = 8, 32, 128, 256, 16
     assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + 256 + S * Hq * C * 4 + S * Hq * 4
                                         + S * Hq * P * D * 4 + S * Hq * P * 4
