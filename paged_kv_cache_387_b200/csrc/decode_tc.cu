@@ -910,20 +910,29 @@ __global__ void __launch_bounds__(THREADS, 2)
                         min(min(MAX_MEMBERS, max(1, NH / G)), a.num_seqs - s))
                   : 1;
       const int sh = grouped ? (int)(wk.y & 0x7ffffffu) : 0;
-      int Lm = 0;  // lane m < members: member m's length and own tiles
-      if (lane < members)
-        Lm = grouped ? effective_len(a.context_lens[s + lane], a.max_context_len, a.max_blocks, B,
-                                     nullptr)
-                     : static_cast<int>(wk.y);
-      const int own_n = lane < members ? max(0, Lm - sh * TILE + TILE - 1) / TILE : 0;
-      int own_incl = own_n;
+      // Lane m < members: member m's length, own tiles and first own tile.
+      // One sequence: its length is the entry's, all its tiles are its own.
+      int Lm, own_n, own_lo, tiles;
+      if (!grouped) {
+        const int L = static_cast<int>(wk.y);
+        tiles = (L + TILE - 1) / TILE;
+        Lm = lane == 0 ? L : 0;
+        own_n = lane == 0 ? tiles : 0;
+        own_lo = 0;
+      } else {
+        Lm = lane < members ? effective_len(a.context_lens[s + lane], a.max_context_len,
+                                            a.max_blocks, B, nullptr)
+                            : 0;
+        own_n = lane < members ? max(0, Lm - sh * TILE + TILE - 1) / TILE : 0;
+        int own_incl = own_n;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(FULL_MASK, own_incl, off);
-        if (lane >= off) own_incl += y;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(FULL_MASK, own_incl, off);
+          if (lane >= off) own_incl += y;
+        }
+        own_lo = sh + own_incl - own_n;
+        tiles = sh + __shfl_sync(FULL_MASK, own_incl, 31);
       }
-      const int own_lo = sh + own_incl - own_n;  // member lane's first own tile
-      const int tiles = sh + __shfl_sync(FULL_MASK, own_incl, 31);
       const int ptg = group_part_tiles(a, grouped, tiles);
       const int tile0 = p * ptg;
       const int n_tiles = max(0, min(tiles, tile0 + ptg) - tile0);
@@ -968,8 +977,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       constexpr int upt = U8 ? 2 : 1;  // table entries per tile
       // All of a lane's table loads are issued before its first store.
       int idv[IDS_PER_LANE];
-      if (members == 1) {  // one sequence: partition tile t is its tile tile0 + t
-        const int L = __shfl_sync(FULL_MASK, Lm, 0);
+      if (!grouped) {  // one sequence: partition tile t is its tile tile0 + t
+        const int L = static_cast<int>(wk.y);
         const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
 #pragma unroll
         for (int k = 0; k < IDS_PER_LANE; ++k) {
