@@ -245,7 +245,6 @@ __device__ __noinline__ void plan_group_round(const DecodeArgs &a, int s, int L,
                                               bool cand, BlockScan block_scan, int &word,
                                               int &gtiles) {
   __shared__ int c_seq[PLAN_THREADS];     // candidate pairs (s-1, s): s
-  __shared__ int c_off[PLAN_THREADS];     // first comparison index of each candidate
   __shared__ int c_mis[PLAN_THREADS];     // first differing block (or the blocks compared)
   __shared__ int g_cnt[PLAN_THREADS];     // members of the group a thread leads
   __shared__ int g_sh[PLAN_THREADS];      // its shared tiles
@@ -254,49 +253,63 @@ __device__ __noinline__ void plan_group_round(const DecodeArgs &a, int s, int L,
   const int tid = threadIdx.x;
   const int S = a.num_seqs, B = a.block_size;
   const int nblk = cand ? (cap * TILE + B - 1) / B : 0;  // blocks covering the span
-  int ncand, work;
-  const int ci = block_scan(cand ? 1 : 0, ncand);
-  const int co = block_scan(cand ? nblk - 1 : 0, work);  // block 0 is already compared
+  int ncand;
+  const int ci = block_scan(cand ? 1 : 0, ncand);  // this candidate's index
   if (cand) {
     c_seq[ci] = s;
-    c_off[ci] = co;
     c_mis[ci] = nblk;
   }
   g_cnt[tid] = 0;
   g_sh[tid] = INT_MAX;
   g_own[tid] = 0;
   __syncthreads();
-  // every comparison of every candidate: f -> (candidate c, block j >= 1).
-  // A thread takes CMP_BATCH consecutive comparisons and issues all their
-  // table loads before it compares, so that their latencies overlap.
-  constexpr int CMP_BATCH = 32;
-  for (int f0 = tid * CMP_BATCH; f0 < work; f0 += PLAN_THREADS * CMP_BATCH) {
-    int lo = 0, hi = ncand - 1;  // the last candidate whose range starts at or before f0
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (c_off[mid] <= f0)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    int c = lo;
-    int cc[CMP_BATCH], jj[CMP_BATCH], va[CMP_BATCH], vb[CMP_BATCH];
+  // Every comparison of every candidate. Warp w takes candidates w, w + 8,
+  // ... in batches of CMP_CANDS; lane l compares blocks 1 + l, 33 + l, ... of
+  // each, CMP_CHUNKS chunks of 32 blocks at a time, with all of a batch's
+  // loads issued before the comparisons. A warp minimum gives the first
+  // differing block.
+  constexpr int NWARP = PLAN_THREADS / 32, CMP_CANDS = 16, CMP_CHUNKS = 2;
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int c0 = warp; c0 < ncand; c0 += NWARP * CMP_CANDS) {
+    const int32_t *rows[CMP_CANDS];
+    int nb[CMP_CANDS], mis[CMP_CANDS];
 #pragma unroll
-    for (int k = 0; k < CMP_BATCH; ++k) {
-      const int f = f0 + k;
-      while (c + 1 < ncand && c_off[c + 1] <= f) ++c;  // the candidate holding f
-      cc[k] = f < work ? c : -1;
-      jj[k] = f - c_off[c] + 1;
-      va[k] = vb[k] = 0;
-      if (f < work) {
-        const int32_t *bt = a.block_tables + (size_t)c_seq[c] * a.max_blocks;
-        va[k] = bt[jj[k]];
-        vb[k] = (bt - a.max_blocks)[jj[k]];
+    for (int k = 0; k < CMP_CANDS; ++k) {
+      const int c = c0 + k * NWARP;
+      rows[k] = a.block_tables + (size_t)(c < ncand ? c_seq[c] : 1) * a.max_blocks;
+      nb[k] = c < ncand ? c_mis[c] : 0;  // blocks covering the candidate's span
+      mis[k] = nb[k];
+    }
+    int longest = 0;
+#pragma unroll
+    for (int k = 0; k < CMP_CANDS; ++k) longest = max(longest, nb[k]);
+    for (int j0 = 1; j0 < longest; j0 += 32 * CMP_CHUNKS) {
+      int va[CMP_CANDS][CMP_CHUNKS], vb[CMP_CANDS][CMP_CHUNKS];
+#pragma unroll
+      for (int k = 0; k < CMP_CANDS; ++k)
+#pragma unroll
+        for (int q = 0; q < CMP_CHUNKS; ++q) {
+          const int j = j0 + lane + 32 * q;
+          const bool in = j < nb[k] && j < mis[k];
+          va[k][q] = in ? rows[k][j] : 0;
+          vb[k][q] = in ? (rows[k] - a.max_blocks)[j] : 0;  // row s-1 precedes row s
+        }
+#pragma unroll
+      for (int k = 0; k < CMP_CANDS; ++k) {
+        int first = mis[k];
+#pragma unroll
+        for (int q = 0; q < CMP_CHUNKS; ++q) {
+          const int j = j0 + lane + 32 * q;
+          if (j < nb[k] && va[k][q] != vb[k][q]) first = min(first, j);
+        }
+        mis[k] = __reduce_min_sync(FULL_MASK, first);
       }
     }
 #pragma unroll
-    for (int k = 0; k < CMP_BATCH; ++k)
-      if (cc[k] >= 0 && va[k] != vb[k]) atomicMin(&c_mis[cc[k]], jj[k]);
+    for (int k = 0; k < CMP_CANDS; ++k) {
+      const int c = c0 + k * NWARP;
+      if (lane == 0 && c < ncand) c_mis[c] = mis[k];
+    }
   }
   __syncthreads();
   const int psh = cand ? min(c_mis[ci] * B / TILE, cap) : 0;
@@ -424,6 +437,7 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   const int newest = a.k_new != nullptr ? 1 : 0;
   bool any_group = false;  // (uniform) a group formed: the words are in a.grp
   int nm = 0;
+  int L1 = 0, word1 = 0, gtiles1 = 0;  // this thread's last pass-1 values
   for (int r0 = 0; r0 < S; r0 += PLAN_THREADS) {
     const int s = r0 + tid;
     int raw = 0, raw_prev = 0;
@@ -459,6 +473,9 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
         a.grp[s] = 0;
       }
     }
+    L1 = L;
+    word1 = word;
+    gtiles1 = gtiles;
     if (s < S) {
       int np, tiles;
       uint32_t w;
@@ -495,8 +512,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     uint32_t word = 0;
     if (s < S) {
       int n, tiles;
-      const int g = any_group ? a.grp[s] : 0;
-      entry_shape(eff_len(s), g, g > 0 ? a.grp_tiles[s] : 0, n, tiles, word);
+      // (one round: this thread's word from pass 1 is still in registers)
+      const int g = !any_group ? 0 : S <= PLAN_THREADS ? word1 : a.grp[s];
+      const int gt = g <= 0 ? 0 : S <= PLAN_THREADS ? gtiles1 : a.grp_tiles[s];
+      entry_shape(S <= PLAN_THREADS ? L1 : eff_len(s), g, gt, n, tiles, word);
       if (n > 1)
         np = n;
       else if (n == 1)
