@@ -336,6 +336,61 @@ __device__ __noinline__ void plan_group_round(const DecodeArgs &a, int s, int L,
   __syncthreads();  // the shared arrays are rewritten by the next round
 }
 
+// The work list of a batch of at most 32 sequences with no shared-prefix
+// groups, built by one warp with shuffles instead of block barriers: the same
+// list plan_kernel builds (lane s holds sequence s).
+__device__ __noinline__ void plan_small(const DecodeArgs &a, int lane) {
+  const int S = a.num_seqs;
+  const int s = lane;
+  int raw = 0, L = 0;
+  if (s < S) {
+    raw = a.context_lens[s];
+    L = effective_len(raw, a.max_context_len, a.max_blocks, a.block_size, nullptr);
+  }
+  const bool bad_len = __any_sync(FULL_MASK, s < S && L < raw);
+  const int pt = max(1, a.part_tokens / TILE);  // tiles per partition
+  const int tiles = (L + TILE - 1) / TILE;
+  const int np = s < S ? max(1, (tiles + pt - 1) / pt) : 0;
+  // region 1: sequences of several partitions, in batch order, each with its
+  // short last partition first
+  const int nm = np > 1 ? np : 0;
+  int incl = nm;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(FULL_MASK, incl, off);
+    if (lane >= off) incl += y;
+  }
+  const int total_m = __shfl_sync(FULL_MASK, incl, 31);
+  uint2 *const list = a.work;
+  if (nm > 0) {
+    const int o = incl - nm;
+    list[o] = make_uint2(pack_pair(s, np - 1), (uint32_t)L);
+    for (int q = 0; q < np - 1; ++q) list[o + 1 + q] = make_uint2(pack_pair(s, q), (uint32_t)L);
+  }
+  // region 2: one-partition sequences, larger size class first, batch order
+  // within a class (a sequence of length 0 is one empty entry)
+  const int bkt = np == 1 ? (PLAN_BUCKETS - 1) -
+                                min(PLAN_BUCKETS - 1, tiles * (PLAN_BUCKETS - 1) / pt)
+                          : INT_MAX;
+  int rank = 0;
+  for (int j = 0; j < 32; ++j) {
+    const int b = __shfl_sync(FULL_MASK, bkt, j);
+    if (b < bkt || (b == bkt && j < lane)) ++rank;
+  }
+  if (np == 1) list[total_m + rank] = make_uint2(pack_pair(s, 0), (uint32_t)L);
+  const int total = total_m + __popc(__ballot_sync(FULL_MASK, np == 1));
+  if (a.merge_cnt) {
+    const int n1 = S * a.num_kv_heads * a.max_chunks;
+    for (int i = lane; i < n1; i += 32) a.merge_cnt[i] = 0;
+    for (int i = lane; i < S * a.num_kv_heads; i += 32) a.merge_cnt2[i] = 0;
+  }
+  if (lane == 0) {
+    a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
+    a.sched[1] = total;
+    if (bad_len) report(a.err, PKV_DEV_CONTEXT_LEN);
+  }
+}
+
 // Build the work list in two regions.
 //  1. Entries of several partitions: all their partitions, entry by entry,
 //     the short last partition first. Their merges then complete while the
@@ -373,6 +428,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int S = a.num_seqs;
   const bool grouping = a.max_group > 1;
+  if (!grouping && S <= 32) {  // a small batch: warp 0 plans alone (no block barriers)
+    if (warp == 0) plan_small(a, lane);
+    return;
+  }
   if (tid < PLAN_BUCKETS) hist[tid] = 0;
   if (tid == 0) bad_len = 0;
   __syncthreads();

@@ -342,3 +342,23 @@ def test_back_to_back_calls_with_changing_batches(fused):
     torch.cuda.synchronize()
     for k, o in outs:
         assert torch.equal(o.view(torch.int16), refs[k].view(torch.int16)), f"batch {k}"
+
+
+@pytest.mark.parametrize("S", [1, 2, 31, 32, 33, 64])
+@pytest.mark.parametrize("part", [0, 64])
+def test_small_batches_plan_paths(S, part):
+    """Up to 32 sequences without shared-prefix groups are planned by one warp,
+    larger batches by the whole plan block: both must give the same work (every
+    partition of every sequence, empty sequences included)."""
+    rng = np.random.default_rng(S + part)
+    lens = rng.integers(0, 300, size=S).tolist()
+    lens[0] = 0
+    if S > 2:
+        lens[1] = 257  # several 64-token partitions
+    c = make_random_case("smallS", 16, 4, 128, 16, lens, torch.bfloat16, seed=S, device=DEV)
+    err = new_err(DEV)
+    got = gpu_decode(c, partition_size=part, err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert (got[0] == 0).all()
+    assert_close_to_oracle(got, oracle_decode(c), torch.bfloat16, f"S{S} p{part}")
