@@ -110,6 +110,43 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
 int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int partition_size);
 
 /*
+ * Decode kernel selection for fp16 / bf16 (a process-wide setting, for tuning
+ * and tests; the results agree within the accuracy bound either way).
+ *
+ * Two kernels implement paged_attn_decode and paged_attn_decode_append:
+ *   - the persistent kernel: a one-CTA plan launch builds a work list from
+ *     context_lens, then two CTAs per SM pull (sequence, partition, KV head)
+ *     items, merging split contexts through the workspace. It balances large
+ *     and ragged batches.
+ *   - the single-wave kernel: when every (sequence, KV head, partition) of
+ *     the call fits in one wave of CTAs, one launch with no plan. CTA
+ *     (p, h, s) attends partition p, and the partitions of one (sequence, KV
+ *     head) form a thread-block cluster (at most 16) whose first CTA merges
+ *     them through distributed shared memory. Contexts of at most 64 tokens
+ *     are attended one warp per (sequence, KV head). The workspace is not
+ *     touched (it is still validated), and shared-prefix grouping does not
+ *     apply. Under PKV_PARTITION_AUTO this kernel chooses its own partition
+ *     length: the most partitions (of at least 64 tokens, at most 16) that
+ *     keep the call within one wave.
+ *
+ * PKV_DISPATCH_AUTO (the default) takes the single-wave kernel whenever the
+ * call fits it, else the persistent one. PKV_DISPATCH_PERSISTENT always takes
+ * the persistent kernel. PKV_DISPATCH_WAVE_CTA never uses the warp-per-item
+ * form. PKV_DISPATCH_WAVE_WARP uses the warp-per-item form for any call with
+ * one partition (partition_size 0, AUTO, or >= the longest context), and
+ * otherwise the persistent kernel.
+ *
+ * Returns the previous mode, or PKV_EINVAL for an unknown mode (the setting
+ * is then unchanged). Safe to call from any thread; calls already issued are
+ * unaffected.
+ */
+#define PKV_DISPATCH_AUTO 0
+#define PKV_DISPATCH_PERSISTENT 1
+#define PKV_DISPATCH_WAVE_CTA 2
+#define PKV_DISPATCH_WAVE_WARP 3
+int pkv_set_decode_dispatch(int mode);
+
+/*
  * paged_attn_decode - one decode step of attention over a paged KV cache.
  *
  * For every sequence s and query head h, with G = num_heads / num_kv_heads,
@@ -135,6 +172,8 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  * num_heads / num_kv_heads is 1 or 2: the whole 16-token tiles of their common
  * leading blocks are read once for all of them. Each sequence still gets its
  * own attention over its own tokens; only the fp32 summation order differs.
+ * (Calls small enough for the single-wave kernel, see pkv_set_decode_dispatch,
+ * attend every sequence alone.)
  *
  * out            [num_seqs][num_heads][head_dim], written entirely. A sequence
  *                with L <= 0 gets zeros. Device memory, or page-locked host
@@ -151,8 +190,9 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  * scale          score multiplier; 1/sqrt(head_dim) gives the usual attention.
  * partition_size tokens per partition. 0 means no split (one partition of
  *                the whole context), PKV_PARTITION_AUTO lets the library
- *                choose (pkv_resolve_partition). Otherwise a positive
- *                multiple of 16.
+ *                choose (pkv_resolve_partition for the persistent kernel; see
+ *                pkv_set_decode_dispatch for the single-wave one). Otherwise
+ *                a positive multiple of 16.
  * workspace      device scratch of at least pkv_decode_workspace_bytes(...)
  *                bytes, 256-byte aligned. Its contents on entry do not
  *                matter. Calls that overlap in time must not share it.

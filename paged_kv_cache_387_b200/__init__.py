@@ -29,10 +29,14 @@ DEV_ERRORS = {1: "block id out of range", 2: "append slot out of range",
 DTYPE_CODES = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 PARTITION_AUTO = -1  # the library picks the partition length from the batch shape
 DEFAULT_PARTITION = PARTITION_AUTO
+# Decode kernel selection (pkv_set_decode_dispatch): the single-wave kernel for
+# calls that fit one wave of CTAs, else the persistent kernel.
+DISPATCH_AUTO, DISPATCH_PERSISTENT, DISPATCH_WAVE_CTA, DISPATCH_WAVE_WARP = 0, 1, 2, 3
 
 EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
            "kv_block_copy", "kv_block_swap", "pkv_check_wait_timeout",
-           "pkv_decode_workspace_bytes", "pkv_resolve_partition", "pkv_status_string")
+           "pkv_decode_workspace_bytes", "pkv_resolve_partition", "pkv_set_decode_dispatch",
+           "pkv_status_string")
 
 
 class PkvError(RuntimeError):
@@ -72,6 +76,8 @@ def load_library():
     lib.pkv_decode_workspace_bytes.restype = Z
     lib.pkv_resolve_partition.argtypes = [I, I, I, I]
     lib.pkv_resolve_partition.restype = I
+    lib.pkv_set_decode_dispatch.argtypes = [I]
+    lib.pkv_set_decode_dispatch.restype = I
     lib.pkv_status_string.argtypes = [I]
     lib.pkv_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -124,6 +130,15 @@ def resolve_partition(num_seqs: int, num_heads: int, max_context_len: int,
     """The partition length a decode call uses (``PARTITION_AUTO`` resolved)."""
     return int(load_library().pkv_resolve_partition(num_seqs, num_heads, max_context_len,
                                                     partition_size))
+
+
+def set_decode_dispatch(mode: int) -> int:
+    """Select the decode kernel for fp16 / bf16 calls, process-wide
+    (``DISPATCH_*``); returns the previous mode."""
+    rc = int(load_library().pkv_set_decode_dispatch(int(mode)))
+    if rc < 0:
+        _check("pkv_set_decode_dispatch", rc)
+    return rc
 
 
 def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "pkv.h"
@@ -75,6 +76,71 @@ bool make_pool_map(CUtensorMap *map, const void *pool, long long rows, int head_
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
 
+// Process-wide decode kernel selection (pkv_set_decode_dispatch).
+std::atomic<int> g_dispatch{PKV_DISPATCH_AUTO};
+
+// Launch shape of a single-wave decode for a 16-bit call, or false when the
+// call does not fit one wave of CTAs (the persistent kernel takes it then).
+//   warp mode: every context fits WAVE_WARP_TILES tiles and one partition;
+//   CTA mode: S * Hkv * P CTAs (P partitions of part_tokens each, P <=
+//     WAVE_MAX_PARTS) are resident at once. Under PKV_PARTITION_AUTO, P is
+//     the most partitions (of at least WAVE_MIN_PART_TILES tiles) that keep
+//     it so.
+bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requested_part,
+               bool *warp_items, int *parts, int *part_tokens) {
+  const int mode = g_dispatch.load(std::memory_order_relaxed);
+  if (mode == PKV_DISPATCH_PERSISTENT) return false;
+  const long long items = (long long)a.num_seqs * a.num_kv_heads;
+  const long long max_len = a.max_context_len;
+  const long long max_tiles = (max_len + 15) / 16;
+  const long long whole = max_tiles > 0 ? max_tiles * 16 : 16;  // one partition holds any context
+  if (whole > 0x7fffffffLL) return false;
+  const bool one_part = auto_part || requested_part == 0 || requested_part >= whole;
+  if (mode != PKV_DISPATCH_WAVE_CTA && one_part &&
+      (max_tiles <= pkv::WAVE_WARP_TILES || mode == PKV_DISPATCH_WAVE_WARP)) {
+    *warp_items = true;
+    *parts = 1;
+    *part_tokens = (int)whole;
+    return true;
+  }
+  if (mode == PKV_DISPATCH_WAVE_WARP) return false;
+  // CTAs (P == 1) or clusters of P CTAs resident at once
+  auto fits = [&](long long P) {
+    int cap = 0;
+    return pkv::decode_wave_capacity(a, dtype, false, (int)P, &cap) == cudaSuccess &&
+           items <= cap;
+  };
+  auto parts_of = [&](long long pt) { return max_len > pt ? (max_len + pt - 1) / pt : 1; };
+  long long P, pt;
+  if (auto_part) {
+    int per_wave = 0;
+    if (pkv::decode_wave_capacity(a, dtype, false, 1, &per_wave) != cudaSuccess) return false;
+    const long long fit = items > 0 ? per_wave / items : 0;
+    const long long by_len = (max_tiles + pkv::WAVE_MIN_PART_TILES - 1) / pkv::WAVE_MIN_PART_TILES;
+    long long want = fit < by_len ? fit : by_len;
+    if (want > pkv::WAVE_MAX_PARTS) want = pkv::WAVE_MAX_PARTS;
+    if (want < 1) want = 1;
+    // Clusters of P CTAs may pack less densely than single CTAs: take fewer
+    // partitions until the cluster shape holds the whole call.
+    for (;; --want) {
+      pt = ((max_len + want - 1) / want + 15) / 16 * 16;
+      if (pt < 16) pt = 16;
+      P = parts_of(pt);
+      if (fits(P)) break;
+      if (want <= 1) return false;
+    }
+  } else {
+    pt = requested_part > 0 ? requested_part : whole;
+    P = parts_of(pt);
+    if (P > pkv::WAVE_MAX_PARTS || !fits(P)) return false;
+  }
+  if (pt > 0x7fffffffLL) return false;
+  *warp_items = false;
+  *parts = (int)P;
+  *part_tokens = (int)pt;
+  return true;
+}
+
 }  // namespace
 
 namespace pkv {
@@ -140,6 +206,11 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
   return (int)part;
 }
 
+int pkv_set_decode_dispatch(int mode) {
+  if (mode < PKV_DISPATCH_AUTO || mode > PKV_DISPATCH_WAVE_WARP) return PKV_EINVAL;
+  return g_dispatch.exchange(mode);
+}
+
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim, int max_context_len,
                                   int partition_size) {
   partition_size = pkv_resolve_partition(num_seqs, num_heads, max_context_len, partition_size);
@@ -162,6 +233,8 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
                 int max_blocks_per_seq, int num_blocks, int max_context_len, float scale,
                 int dtype, int partition_size, void *workspace, size_t workspace_bytes,
                 int32_t *err, void *stream, const void *k_new, const void *v_new) {
+  const bool auto_part = partition_size == PKV_PARTITION_AUTO;
+  const int requested_part = partition_size;
   partition_size = pkv_resolve_partition(num_seqs, num_heads, max_context_len, partition_size);
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0 || max_context_len < 0 ||
@@ -247,6 +320,15 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
     if (!make_pool_map(&tmK, k_pool, rows, head_dim, a.unit8 != 0) ||
         !make_pool_map(&tmV, v_pool, rows, head_dim, a.unit8 != 0))
       return PKV_ECUDA;
+    // A call that fits one wave of CTAs: one launch, no plan, no workspace.
+    bool warp_items = false;
+    int wparts = 1, wtokens = 0;
+    if (plan_wave(a, dtype, auto_part, requested_part, &warp_items, &wparts, &wtokens)) {
+      pkv::DecodeArgs b = a;
+      b.part_tokens = wtokens;
+      b.max_parts = wparts;
+      return cuda_status(pkv::launch_decode_wave(b, dtype, warp_items, wparts, tmK, tmV, st));
+    }
     // plan + decode; the partition merge is fused into the decode kernel
     return cuda_status(pkv::launch_decode_tc(a, dtype, tmK, tmV, st));
   }

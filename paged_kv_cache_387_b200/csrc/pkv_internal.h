@@ -56,6 +56,15 @@ struct DecodeArgs {
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
 
+// Single-wave decode (decode_wave.cu): at most this many partitions per
+// (sequence, KV head), one thread-block cluster of that many CTAs.
+constexpr int WAVE_MAX_PARTS = 16;
+// Contexts of at most this many 16-token tiles are attended one warp each.
+constexpr int WAVE_WARP_TILES = 4;
+// Under PKV_PARTITION_AUTO a single-wave partition holds at least this many
+// tiles (one per warp).
+constexpr int WAVE_MIN_PART_TILES = 4;
+
 // Decode workspace, in order: scheduling words (256 B), the work list, the
 // per-sequence group words (two int32 per sequence), then
 // (only when a context can span several partitions) the merge counters, the
@@ -72,6 +81,16 @@ cudaError_t launch_wait_timeout_probe(long long limit_cycles, int32_t *err, cuda
 cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &tmK,
                              const CUtensorMap &tmV, cudaStream_t stream);
 cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream);
+// Single-wave decode for fp16 / bf16: `parts` partitions of a.part_tokens
+// tokens per (sequence, KV head), or with warp_items one warp per (sequence,
+// KV head) and one partition. The workspace is not used.
+cudaError_t launch_decode_wave(const DecodeArgs &a, int dtype, bool warp_items, int parts,
+                               const CUtensorMap &tmK, const CUtensorMap &tmV,
+                               cudaStream_t stream);
+// How much of that work one wave holds: CTAs (warp_items, or parts == 1), or
+// clusters of `parts` CTAs. 0 when the cluster shape cannot be resident.
+cudaError_t decode_wave_capacity(const DecodeArgs &a, int dtype, bool warp_items, int parts,
+                                 int *cap);
 cudaError_t launch_merge(const DecodeArgs &a, int dtype, cudaStream_t stream);
 
 cudaError_t launch_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,

@@ -18,6 +18,16 @@ DEV = "cuda"
 TIMEOUT = 5  # PKV_DEV_WAIT_TIMEOUT
 
 
+@pytest.fixture(autouse=True, params=["auto", "persistent"])
+def _dispatch(request):
+    """Both decode kernels: the single-wave one (these calls are small) and
+    the persistent one."""
+    if request.param == "persistent":
+        pkv.set_decode_dispatch(pkv.DISPATCH_PERSISTENT)
+    yield
+    pkv.set_decode_dispatch(pkv.DISPATCH_AUTO)
+
+
 def test_bounded_wait_gives_up_and_reports():
     err = new_err(DEV)
     t0 = time.time()

@@ -15,6 +15,16 @@ DEV = "cuda"
 DT = {"f16": torch.float16, "bf16": torch.bfloat16}
 
 
+@pytest.fixture(autouse=True, params=["auto", "persistent"])
+def _dispatch(request):
+    """Every test runs under the default kernel selection (small calls take the
+    single-wave kernel) and with the persistent kernel forced."""
+    if request.param == "persistent":
+        pkv.set_decode_dispatch(pkv.DISPATCH_PERSISTENT)
+    yield
+    pkv.set_decode_dispatch(pkv.DISPATCH_AUTO)
+
+
 def fused_vs_oracle(c, part, what):
     kc, vc = c.k_pool.cpu(), c.v_pool.cpu()
     oracle.cache_append(kc, vc, c.k_new.cpu(), c.v_new.cpu(), c.slot_mapping.cpu())

@@ -16,6 +16,16 @@ DEV = "cuda"
 DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
 
 
+@pytest.fixture(autouse=True, params=["auto", "persistent"])
+def _dispatch(request):
+    """Every test runs under the default kernel selection (small calls take the
+    single-wave kernel) and with the persistent kernel forced."""
+    if request.param == "persistent":
+        pkv.set_decode_dispatch(pkv.DISPATCH_PERSISTENT)
+    yield
+    pkv.set_decode_dispatch(pkv.DISPATCH_AUTO)
+
+
 # ---------------------------------------------------------------------------
 # decode: small cases spanning several tiles and a ragged tail
 # ---------------------------------------------------------------------------
