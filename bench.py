@@ -79,6 +79,11 @@ def parse_args():
     ap.add_argument("--separate-append", action="store_true",
                     help="run kv_cache_append and paged_attn_decode as two calls instead of "
                          "the fused paged_attn_decode_append")
+    ap.add_argument("--small-batch-only", action="store_true",
+                    help="time only the small calls (the line's small_batch entry) on one GPU "
+                         "and print them")
+    ap.add_argument("--small-batch-shapes", default=None,
+                    help="comma-separated subset of the small calls, e.g. 1x4096,256x16")
     return ap.parse_args()
 
 
@@ -537,6 +542,84 @@ def time_fused_call(pkv, case, steps, warmup, stream):
     return a.elapsed_time(b) / steps
 
 
+# Small calls: Llama-8B heads (32 query / 8 KV, d128), bf16, 16-token blocks,
+# one step of the fused append + decode with PARTITION_AUTO.
+SMALL_BATCHES = {"1x16": [16], "1x4096": [4096], "1x8192": [8192], "4x16384": [16384] * 4,
+                 "32x1024": [1024] * 32, "256x16": [16] * 256}
+
+
+def small_batch_lines(pkv, dev, stream, shapes=None):
+    """Device microseconds per small call, under the default kernel selection
+    (these calls take the single-wave kernel) and with the persistent kernel
+    forced:
+      graph_us: 50 back-to-back calls replayed from a CUDA graph, per call
+        (the K/V, 0.5-134 MB, stays in the 126 MB L2 when it fits);
+      cold_us: one call after a 256 MB write has evicted L2, timed by events
+        around it (median of 15), with its K/V GB/s."""
+    import torch
+    from pkv_inputs import make_random_case
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    try:
+        for name, lens in SMALL_BATCHES.items():
+            if shapes and name not in shapes:
+                continue
+            c = make_random_case("small_" + name, 32, 8, 128, 16, lens, torch.bfloat16, seed=1,
+                                 device=dev, with_append=True)
+            mcl = c.max_context_len
+            out = torch.empty_like(c.q)
+            wsb = pkv.decode_workspace_bytes(c.num_seqs, c.num_heads, c.head_dim, mcl,
+                                             pkv.PARTITION_AUTO)
+            ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+            kv_bytes = int(c.context_lens.sum()) * 8 * 128 * 2 * 2
+
+            def call(st):
+                pkv.paged_attn_decode_append(out, c.q, c.k_new, c.v_new, c.k_pool, c.v_pool,
+                                             c.block_tables, c.context_lens, c.scale, mcl,
+                                             partition_size=pkv.PARTITION_AUTO, workspace=ws,
+                                             stream=st)
+            entry = {"kv_bytes": kv_bytes}
+            for mode, key in ((pkv.DISPATCH_AUTO, "single_wave"),
+                              (pkv.DISPATCH_PERSISTENT, "persistent")):
+                pkv.set_decode_dispatch(mode)
+                for _ in range(5):
+                    call(stream)
+                torch.cuda.synchronize()
+                cap = torch.cuda.Stream(device=dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+                    for _ in range(50):
+                        call(cap)
+                g.replay()
+                torch.cuda.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                torch.cuda.synchronize()
+                graph_us = a.elapsed_time(b) / 50 * 1e3
+                del g
+                cold = []
+                for i in range(15):
+                    flush.fill_(i & 0xff)
+                    a.record(stream)
+                    call(stream)
+                    b.record(stream)
+                    b.synchronize()
+                    cold.append(a.elapsed_time(b) * 1e3)
+                cold_us = statistics.median(cold)
+                entry[key] = {"graph_us": graph_us, "cold_us": cold_us,
+                              "cold_kv_GB/s": kv_bytes / (cold_us * 1e-6) / 1e9}
+            res[name] = entry
+            del c, out, ws
+    finally:
+        pkv.set_decode_dispatch(pkv.DISPATCH_AUTO)
+    del flush
+    torch.cuda.empty_cache()
+    return {"shape": "32 query / 8 KV heads, d128, bf16, block 16, fused append, "
+                     "PARTITION_AUTO", "calls": res}
+
+
 def extra_lines(args, dev, rank, pkv, stream, peak):
     """The other workloads of the scope, each timed on the device like the
     headline (the fused append + decode call, `--steps` calls after
@@ -570,6 +653,7 @@ def extra_lines(args, dev, rank, pkv, stream, peak):
         lines[w] = d
         del case
         torch.cuda.empty_cache()
+    lines["small_batch"] = small_batch_lines(pkv, dev, stream)
     return lines
 
 
@@ -945,6 +1029,18 @@ def main():
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return
+    if args.small_batch_only:
+        import torch
+        import paged_kv_cache_387_b200 as pkv
+        from paged_kv_cache_387_b200 import build as pkv_build
+        pkv_build.build()
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        shapes = args.small_batch_shapes.split(",") if args.small_batch_shapes else None
+        if rank == 0:
+            print(json.dumps({"small_batch": small_batch_lines(
+                pkv, dev, torch.cuda.current_stream(dev), shapes)}), flush=True)
         return
     import torch
     import torch.distributed as dist
