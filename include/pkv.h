@@ -129,11 +129,17 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  *     length: the most partitions (of at least 64 tokens, at most 16) that
  *     keep the call within one wave.
  *
+ * A single-wave CTA has 4 warps, or 8 when the call has at most one CTA per
+ * SM and every warp gets at least two 16-token tiles (so that each SM
+ * sub-partition still runs two warps).
+ *
  * PKV_DISPATCH_AUTO (the default) takes the single-wave kernel whenever the
  * call fits it, else the persistent one. PKV_DISPATCH_PERSISTENT always takes
  * the persistent kernel. PKV_DISPATCH_WAVE_CTA never uses the warp-per-item
- * form. PKV_DISPATCH_WAVE_WARP uses the warp-per-item form for any call with
- * one partition (partition_size 0, AUTO, or >= the longest context), and
+ * form and keeps CTAs at 4 warps; PKV_DISPATCH_WAVE_CTA8 never uses the
+ * warp-per-item form and takes 8-warp CTAs whenever they fit one per SM.
+ * PKV_DISPATCH_WAVE_WARP uses the warp-per-item form for any call with one
+ * partition (partition_size 0, AUTO, or >= the longest context), and
  * otherwise the persistent kernel.
  *
  * Returns the previous mode, or PKV_EINVAL for an unknown mode (the setting
@@ -144,6 +150,7 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
 #define PKV_DISPATCH_PERSISTENT 1
 #define PKV_DISPATCH_WAVE_CTA 2
 #define PKV_DISPATCH_WAVE_WARP 3
+#define PKV_DISPATCH_WAVE_CTA8 4
 int pkv_set_decode_dispatch(int mode);
 
 /*

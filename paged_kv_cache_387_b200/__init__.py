@@ -32,6 +32,7 @@ DEFAULT_PARTITION = PARTITION_AUTO
 # Decode kernel selection (pkv_set_decode_dispatch): the single-wave kernel for
 # calls that fit one wave of CTAs, else the persistent kernel.
 DISPATCH_AUTO, DISPATCH_PERSISTENT, DISPATCH_WAVE_CTA, DISPATCH_WAVE_WARP = 0, 1, 2, 3
+DISPATCH_WAVE_CTA8 = 4
 
 EXPORTS = ("paged_attn_decode", "paged_attn_decode_append", "kv_cache_append",
            "kv_block_copy", "kv_block_swap", "pkv_check_wait_timeout",

@@ -85,9 +85,10 @@ std::atomic<int> g_dispatch{PKV_DISPATCH_AUTO};
 //   CTA mode: S * Hkv * P CTAs (P partitions of part_tokens each, P <=
 //     WAVE_MAX_PARTS) are resident at once. Under PKV_PARTITION_AUTO, P is
 //     the most partitions (of at least WAVE_MIN_PART_TILES tiles) that keep
-//     it so.
+//     it so. CTAs of 8 warps when they are at most one per SM and every warp
+//     gets at least two tiles, else 4.
 bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requested_part,
-               bool *warp_items, int *parts, int *part_tokens) {
+               bool *warp_items, int *warps, int *parts, int *part_tokens) {
   const int mode = g_dispatch.load(std::memory_order_relaxed);
   if (mode == PKV_DISPATCH_PERSISTENT) return false;
   const long long items = (long long)a.num_seqs * a.num_kv_heads;
@@ -96,25 +97,26 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
   const long long whole = max_tiles > 0 ? max_tiles * 16 : 16;  // one partition holds any context
   if (whole > 0x7fffffffLL) return false;
   const bool one_part = auto_part || requested_part == 0 || requested_part >= whole;
-  if (mode != PKV_DISPATCH_WAVE_CTA && one_part &&
+  if (mode != PKV_DISPATCH_WAVE_CTA && mode != PKV_DISPATCH_WAVE_CTA8 && one_part &&
       (max_tiles <= pkv::WAVE_WARP_TILES || mode == PKV_DISPATCH_WAVE_WARP)) {
     *warp_items = true;
+    *warps = 4;
     *parts = 1;
     *part_tokens = (int)whole;
     return true;
   }
   if (mode == PKV_DISPATCH_WAVE_WARP) return false;
   // CTAs (P == 1) or clusters of P CTAs resident at once
-  auto fits = [&](long long P) {
+  auto fits = [&](long long P, int nw) {
     int cap = 0;
-    return pkv::decode_wave_capacity(a, dtype, false, (int)P, &cap) == cudaSuccess &&
+    return pkv::decode_wave_capacity(a, dtype, false, nw, (int)P, &cap) == cudaSuccess &&
            items <= cap;
   };
   auto parts_of = [&](long long pt) { return max_len > pt ? (max_len + pt - 1) / pt : 1; };
   long long P, pt;
   if (auto_part) {
     int per_wave = 0;
-    if (pkv::decode_wave_capacity(a, dtype, false, 1, &per_wave) != cudaSuccess) return false;
+    if (pkv::decode_wave_capacity(a, dtype, false, 4, 1, &per_wave) != cudaSuccess) return false;
     const long long fit = items > 0 ? per_wave / items : 0;
     const long long by_len = (max_tiles + pkv::WAVE_MIN_PART_TILES - 1) / pkv::WAVE_MIN_PART_TILES;
     long long want = fit < by_len ? fit : by_len;
@@ -126,16 +128,44 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
       pt = ((max_len + want - 1) / want + 15) / 16 * 16;
       if (pt < 16) pt = 16;
       P = parts_of(pt);
-      if (fits(P)) break;
+      if (fits(P, 4)) break;
       if (want <= 1) return false;
     }
   } else {
     pt = requested_part > 0 ? requested_part : whole;
     P = parts_of(pt);
-    if (P > pkv::WAVE_MAX_PARTS || !fits(P)) return false;
+    if (P > pkv::WAVE_MAX_PARTS || !fits(P, 4)) return false;
   }
   if (pt > 0x7fffffffLL) return false;
+  // 8-warp CTAs: at most one per SM, every warp with two tiles or more.
+  int nw = 4;
+  int per_wave8 = 0;  // 8-warp CTAs resident at once
+  if (mode != PKV_DISPATCH_WAVE_CTA &&
+      pkv::decode_wave_capacity(a, dtype, false, 8, 1, &per_wave8) == cudaSuccess) {
+    auto fits8 = [&](long long P8, long long pt8) {
+      return items * P8 <= per_wave8 && (mode == PKV_DISPATCH_WAVE_CTA8 || pt8 / 16 >= 16) &&
+             (P8 == 1 || fits(P8, 8));
+    };
+    if (auto_part) {
+      // As many warps or more in 8-warp CTAs: from P down to P / 2 partitions
+      // (a cluster of 8-warp CTAs spans twice the SMs, so fewer fit a GPC).
+      for (long long want = P; want >= 1 && 2 * want >= P; --want) {
+        long long pt8 = ((max_len + want - 1) / want + 15) / 16 * 16;
+        if (pt8 < 16) pt8 = 16;
+        const long long P8 = parts_of(pt8);
+        if (fits8(P8, pt8)) {
+          nw = 8;
+          P = P8;
+          pt = pt8;
+          break;
+        }
+      }
+    } else if (fits8(P, pt)) {
+      nw = 8;
+    }
+  }
   *warp_items = false;
+  *warps = nw;
   *parts = (int)P;
   *part_tokens = (int)pt;
   return true;
@@ -207,7 +237,7 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
 }
 
 int pkv_set_decode_dispatch(int mode) {
-  if (mode < PKV_DISPATCH_AUTO || mode > PKV_DISPATCH_WAVE_WARP) return PKV_EINVAL;
+  if (mode < PKV_DISPATCH_AUTO || mode > PKV_DISPATCH_WAVE_CTA8) return PKV_EINVAL;
   return g_dispatch.exchange(mode);
 }
 
@@ -322,12 +352,13 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
       return PKV_ECUDA;
     // A call that fits one wave of CTAs: one launch, no plan, no workspace.
     bool warp_items = false;
-    int wparts = 1, wtokens = 0;
-    if (plan_wave(a, dtype, auto_part, requested_part, &warp_items, &wparts, &wtokens)) {
+    int wwarps = 4, wparts = 1, wtokens = 0;
+    if (plan_wave(a, dtype, auto_part, requested_part, &warp_items, &wwarps, &wparts, &wtokens)) {
       pkv::DecodeArgs b = a;
       b.part_tokens = wtokens;
       b.max_parts = wparts;
-      return cuda_status(pkv::launch_decode_wave(b, dtype, warp_items, wparts, tmK, tmV, st));
+      return cuda_status(
+          pkv::launch_decode_wave(b, dtype, warp_items, wwarps, wparts, tmK, tmV, st));
     }
     // plan + decode; the partition merge is fused into the decode kernel
     return cuda_status(pkv::launch_decode_tc(a, dtype, tmK, tmV, st));

@@ -1361,8 +1361,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         len = L0;
         valid = min(TILE, L0 - tok0);
         mem = 0;
-        use0 = col0_live;
-        use1 = col1_live;
+        use0 = true;  // columns past the G heads hold zero queries and are never combined
+        use1 = true;
         has_new = j == j_new;
       } else {
         const TileLoc loc = locate_tile<Shape::GROUPS>(view, tile0 + tile_idx, lane);

@@ -47,39 +47,44 @@ namespace pkv {
 namespace {
 
 constexpr int WV_TILE = 16;                // tokens per tile
-constexpr int WV_WARPS = 4;                // warps per CTA, all of them consumers
-constexpr int WV_THREADS = WV_WARPS * 32;
+// Warps per CTA, all of them consumers: 4 (two CTAs per SM at head_dim 128),
+// or 8 when the call has at most one CTA per SM, so that each SM sub-partition
+// still runs two warps.
 constexpr int WV_HALF = WV_TILE * 128;     // one 64-element box of a tile: 16 rows x 128 B
 constexpr int WV_BOX_COLS = 64;
 constexpr int WV_COLS = 8;                 // score columns of the MMA: query heads of a KV head
 constexpr float WV_SLACK = 8.f;            // lazy max: rescale only past 2^8 growth
 
-template <int D>
+template <int D, int NW>
 struct WaveShape {
+  static constexpr int THREADS = NW * 32;
   static constexpr int HALVES = D / WV_BOX_COLS;
   static constexpr int KT_BYTES = HALVES * WV_HALF;  // one K (or V) tile
   static constexpr int STAGE_BYTES = 2 * KT_BYTES;   // K + V
   static constexpr int NSTAGE = 3;
-  static constexpr int RING_BYTES = WV_WARPS * NSTAGE * STAGE_BYTES;
+  static constexpr int RING_BYTES = NW * NSTAGE * STAGE_BYTES;
   // After the tiles, the ring is reused: the warps' combine rows, the CTA's
   // partial result, then the merge weights.
   static constexpr int AS = D + 4;  // padded combine row (floats)
   static constexpr int CW_FLOATS = WV_COLS * AS + 2 * WV_COLS;  // acc[8][D+4], m[8], l[8]
-  static constexpr int PART_OFF = (WV_WARPS * CW_FLOATS * 4 + 15) & ~15;
+  static constexpr int PART_OFF = (NW * CW_FLOATS * 4 + 15) & ~15;
   static constexpr int PART_LSE_OFF = PART_OFF + WV_COLS * D * 4;
   static constexpr int WTS_OFF = PART_LSE_OFF + WV_COLS * 4;
   static constexpr int WTS_FLOATS = WV_COLS * WAVE_MAX_PARTS;  // >= the combine's [8][4] + [8]
   static constexpr int BAR_OFF = RING_BYTES;
-  static constexpr int SMEM_BYTES = RING_BYTES + WV_WARPS * NSTAGE * 8 + 1024;  // + alignment
+  static constexpr int SMEM_BYTES = RING_BYTES + NW * NSTAGE * 8 + 1024;  // + alignment
   static_assert(WTS_OFF + WTS_FLOATS * 4 <= RING_BYTES, "combine areas fit in the ring");
-  static_assert(WTS_FLOATS >= WV_COLS * WV_WARPS + WV_COLS, "scales fit in the weights area");
+  static_assert(WTS_FLOATS >= WV_COLS * NW + WV_COLS, "scales fit in the weights area");
+  static_assert(SMEM_BYTES <= 227 * 1024, "one CTA fits an SM");
 };
 
-template <typename T, int D, bool U8, bool WARP_ITEMS>
-__global__ void __launch_bounds__(WV_THREADS, 2)
+template <typename T, int D, bool U8, bool WARP_ITEMS, int NW>
+__global__ void __launch_bounds__(NW * 32, 8 / NW)
     decode_wave_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const DecodeArgs a) {
-  using Shape = WaveShape<D>;
+  using Shape = WaveShape<D, NW>;
+  constexpr int WV_WARPS = NW;
+  constexpr int WV_THREADS = Shape::THREADS;
   constexpr int NSTAGE = Shape::NSTAGE;
   constexpr int AS = Shape::AS;
   constexpr int CH = D / 8;  // 16-byte chunks per K or V row
@@ -533,7 +538,7 @@ std::mutex g_wave_mu;
 std::map<std::tuple<int, const void *, int>, int> g_wave_cache;
 
 template <typename Kern>
-cudaError_t cached_capacity(Kern kern, int smem, int cluster, int dev, int *out) {
+cudaError_t cached_capacity(Kern kern, int smem, int threads, int cluster, int dev, int *out) {
   const auto key = std::make_tuple(dev, reinterpret_cast<const void *>(kern), cluster);
   {
     std::lock_guard<std::mutex> lock(g_wave_mu);
@@ -548,7 +553,7 @@ cudaError_t cached_capacity(Kern kern, int smem, int cluster, int dev, int *out)
   int v = 0;
   if (cluster <= 1) {
     int per_sm = 0, sms = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, WV_THREADS, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -558,7 +563,7 @@ cudaError_t cached_capacity(Kern kern, int smem, int cluster, int dev, int *out)
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)cluster, 1, 1);
-    cfg.blockDim = dim3(WV_THREADS);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -579,21 +584,23 @@ cudaError_t cached_capacity(Kern kern, int smem, int cluster, int dev, int *out)
   return cudaSuccess;
 }
 
-template <typename T, int D, bool U8, bool WI>
+template <typename T, int D, bool U8, bool WI, int NW>
 cudaError_t wave_capacity_t(int cluster, int *out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  return cached_capacity(decode_wave_kernel<T, D, U8, WI>, WaveShape<D>::SMEM_BYTES, cluster,
-                         dev, out);
+  using Shape = WaveShape<D, NW>;
+  return cached_capacity(decode_wave_kernel<T, D, U8, WI, NW>, Shape::SMEM_BYTES, Shape::THREADS,
+                         cluster, dev, out);
 }
 
-template <typename T, int D, bool U8, bool WI>
+template <typename T, int D, bool U8, bool WI, int NW>
 cudaError_t launch_wave_t(const DecodeArgs &a, int parts, const CUtensorMap &tmK,
                           const CUtensorMap &tmV, cudaStream_t stream) {
-  auto kern = decode_wave_kernel<T, D, U8, WI>;
+  using Shape = WaveShape<D, NW>;
+  auto kern = decode_wave_kernel<T, D, U8, WI, NW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       WaveShape<D>::SMEM_BYTES);
+                                       Shape::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   if (!WI && parts > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -602,12 +609,12 @@ cudaError_t launch_wave_t(const DecodeArgs &a, int parts, const CUtensorMap &tmK
   cudaLaunchConfig_t cfg = {};
   if (WI) {
     const long long items = (long long)a.num_seqs * a.num_kv_heads;
-    cfg.gridDim = dim3((unsigned)((items + WV_WARPS - 1) / WV_WARPS));
+    cfg.gridDim = dim3((unsigned)((items + NW - 1) / NW));
   } else {
     cfg.gridDim = dim3((unsigned)parts, (unsigned)a.num_kv_heads, (unsigned)a.num_seqs);
   }
-  cfg.blockDim = dim3(WV_THREADS);
-  cfg.dynamicSmemBytes = WaveShape<D>::SMEM_BYTES;
+  cfg.blockDim = dim3(Shape::THREADS);
+  cfg.dynamicSmemBytes = Shape::SMEM_BYTES;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -625,45 +632,58 @@ cudaError_t launch_wave_t(const DecodeArgs &a, int parts, const CUtensorMap &tmK
   return cudaLaunchKernelEx(&cfg, kern, tmK, tmV, a);
 }
 
-template <typename T, bool U8, bool WI>
+template <typename T, bool U8, bool WI, int NW>
 cudaError_t wave_dispatch_d(bool launch, const DecodeArgs &a, int parts, const CUtensorMap *tmK,
                             const CUtensorMap *tmV, cudaStream_t stream, int *cap) {
   if (a.head_dim == 64)
-    return launch ? launch_wave_t<T, 64, U8, WI>(a, parts, *tmK, *tmV, stream)
-                  : wave_capacity_t<T, 64, U8, WI>(WI ? 1 : parts, cap);
-  return launch ? launch_wave_t<T, 128, U8, WI>(a, parts, *tmK, *tmV, stream)
-                : wave_capacity_t<T, 128, U8, WI>(WI ? 1 : parts, cap);
+    return launch ? launch_wave_t<T, 64, U8, WI, NW>(a, parts, *tmK, *tmV, stream)
+                  : wave_capacity_t<T, 64, U8, WI, NW>(WI ? 1 : parts, cap);
+  return launch ? launch_wave_t<T, 128, U8, WI, NW>(a, parts, *tmK, *tmV, stream)
+                : wave_capacity_t<T, 128, U8, WI, NW>(WI ? 1 : parts, cap);
+}
+
+// Warp form: 4 warps per CTA. CTA form: 4 or 8 warps.
+template <typename T, bool U8>
+cudaError_t wave_dispatch_u(bool launch, const DecodeArgs &a, bool warp_items, int warps,
+                            int parts, const CUtensorMap *tmK, const CUtensorMap *tmV,
+                            cudaStream_t stream, int *cap) {
+  if (warp_items)
+    return wave_dispatch_d<T, U8, true, 4>(launch, a, parts, tmK, tmV, stream, cap);
+  if (warps == 8)
+    return wave_dispatch_d<T, U8, false, 8>(launch, a, parts, tmK, tmV, stream, cap);
+  return wave_dispatch_d<T, U8, false, 4>(launch, a, parts, tmK, tmV, stream, cap);
 }
 
 template <typename T>
-cudaError_t wave_dispatch(bool launch, const DecodeArgs &a, bool warp_items, int parts,
+cudaError_t wave_dispatch(bool launch, const DecodeArgs &a, bool warp_items, int warps, int parts,
                           const CUtensorMap *tmK, const CUtensorMap *tmV, cudaStream_t stream,
                           int *cap) {
-  if (a.unit8)
-    return warp_items ? wave_dispatch_d<T, true, true>(launch, a, parts, tmK, tmV, stream, cap)
-                      : wave_dispatch_d<T, true, false>(launch, a, parts, tmK, tmV, stream, cap);
-  return warp_items ? wave_dispatch_d<T, false, true>(launch, a, parts, tmK, tmV, stream, cap)
-                    : wave_dispatch_d<T, false, false>(launch, a, parts, tmK, tmV, stream, cap);
+  return a.unit8 ? wave_dispatch_u<T, true>(launch, a, warp_items, warps, parts, tmK, tmV, stream,
+                                            cap)
+                 : wave_dispatch_u<T, false>(launch, a, warp_items, warps, parts, tmK, tmV,
+                                             stream, cap);
 }
 
 }  // namespace
 
-cudaError_t decode_wave_capacity(const DecodeArgs &a, int dtype, bool warp_items, int parts,
-                                 int *cap) {
+cudaError_t decode_wave_capacity(const DecodeArgs &a, int dtype, bool warp_items, int warps,
+                                 int parts, int *cap) {
   *cap = 0;
   return dtype == PKV_BF16
-             ? wave_dispatch<__nv_bfloat16>(false, a, warp_items, parts, nullptr, nullptr,
+             ? wave_dispatch<__nv_bfloat16>(false, a, warp_items, warps, parts, nullptr, nullptr,
                                             nullptr, cap)
-             : wave_dispatch<__half>(false, a, warp_items, parts, nullptr, nullptr, nullptr, cap);
+             : wave_dispatch<__half>(false, a, warp_items, warps, parts, nullptr, nullptr,
+                                     nullptr, cap);
 }
 
-cudaError_t launch_decode_wave(const DecodeArgs &a, int dtype, bool warp_items, int parts,
-                               const CUtensorMap &tmK, const CUtensorMap &tmV,
+cudaError_t launch_decode_wave(const DecodeArgs &a, int dtype, bool warp_items, int warps,
+                               int parts, const CUtensorMap &tmK, const CUtensorMap &tmV,
                                cudaStream_t stream) {
   return dtype == PKV_BF16
-             ? wave_dispatch<__nv_bfloat16>(true, a, warp_items, parts, &tmK, &tmV, stream,
+             ? wave_dispatch<__nv_bfloat16>(true, a, warp_items, warps, parts, &tmK, &tmV, stream,
                                             nullptr)
-             : wave_dispatch<__half>(true, a, warp_items, parts, &tmK, &tmV, stream, nullptr);
+             : wave_dispatch<__half>(true, a, warp_items, warps, parts, &tmK, &tmV, stream,
+                                     nullptr);
 }
 
 }  // namespace pkv

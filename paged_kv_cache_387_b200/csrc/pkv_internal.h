@@ -82,15 +82,16 @@ cudaError_t launch_decode_tc(const DecodeArgs &a, int dtype, const CUtensorMap &
                              const CUtensorMap &tmV, cudaStream_t stream);
 cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream);
 // Single-wave decode for fp16 / bf16: `parts` partitions of a.part_tokens
-// tokens per (sequence, KV head), or with warp_items one warp per (sequence,
-// KV head) and one partition. The workspace is not used.
-cudaError_t launch_decode_wave(const DecodeArgs &a, int dtype, bool warp_items, int parts,
-                               const CUtensorMap &tmK, const CUtensorMap &tmV,
+// tokens per (sequence, KV head) on CTAs of `warps` (4 or 8) warps, or with
+// warp_items one warp per (sequence, KV head) and one partition (4-warp
+// CTAs). The workspace is not used.
+cudaError_t launch_decode_wave(const DecodeArgs &a, int dtype, bool warp_items, int warps,
+                               int parts, const CUtensorMap &tmK, const CUtensorMap &tmV,
                                cudaStream_t stream);
 // How much of that work one wave holds: CTAs (warp_items, or parts == 1), or
 // clusters of `parts` CTAs. 0 when the cluster shape cannot be resident.
-cudaError_t decode_wave_capacity(const DecodeArgs &a, int dtype, bool warp_items, int parts,
-                                 int *cap);
+cudaError_t decode_wave_capacity(const DecodeArgs &a, int dtype, bool warp_items, int warps,
+                                 int parts, int *cap);
 cudaError_t launch_merge(const DecodeArgs &a, int dtype, cudaStream_t stream);
 
 cudaError_t launch_append(void *k_pool, void *v_pool, const void *k_new, const void *v_new,

@@ -50,6 +50,8 @@ def decode_ws(c, part, ws, err=None, fused=False):
 def test_dispatch_setting_round_trips(dispatch):
     assert pkv.set_decode_dispatch(pkv.DISPATCH_PERSISTENT) == pkv.DISPATCH_AUTO
     assert pkv.set_decode_dispatch(pkv.DISPATCH_WAVE_CTA) == pkv.DISPATCH_PERSISTENT
+    assert pkv.set_decode_dispatch(pkv.DISPATCH_WAVE_CTA8) == pkv.DISPATCH_WAVE_CTA
+    assert pkv.set_decode_dispatch(pkv.DISPATCH_WAVE_CTA) == pkv.DISPATCH_WAVE_CTA8
     with pytest.raises(pkv.PkvError):
         pkv.set_decode_dispatch(7)
     assert pkv.set_decode_dispatch(pkv.DISPATCH_AUTO) == pkv.DISPATCH_WAVE_CTA
@@ -79,8 +81,11 @@ def test_wave_leaves_workspace_untouched(dispatch, lens, part):
 @pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 8), (64, 24)])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (32, 8), (8, 1), (6, 2)])
 @pytest.mark.parametrize("nparts", [2, 3, 9, 16])
-def test_cluster_partitions_match_oracle(dt, D, B, Hq, Hkv, nparts, dispatch):
-    dispatch(pkv.DISPATCH_WAVE_CTA)
+@pytest.mark.parametrize("mode", [pkv.DISPATCH_WAVE_CTA, pkv.DISPATCH_WAVE_CTA8])
+def test_cluster_partitions_match_oracle(dt, D, B, Hq, Hkv, nparts, mode, dispatch):
+    """4-warp CTAs, and 8-warp CTAs (at most one CTA per SM: these calls stay
+    well below it)."""
+    dispatch(mode)
     part = 128
     lens = [nparts * part, nparts * part - 17, (nparts - 1) * part + 1, 1, 0, 77]
     lens = lens[:max(1, min(len(lens), 120 // (Hkv * nparts)))]  # well inside one wave
@@ -142,7 +147,7 @@ def test_auto_partition_single_wave(dt, lens):
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16"])
-@pytest.mark.parametrize("mode", ["cta", "warp"])
+@pytest.mark.parametrize("mode", ["cta", "cta8", "warp"])
 @pytest.mark.parametrize("D,B", [(128, 16), (64, 32), (128, 8)])
 def test_fused_append_single_wave(dt, mode, D, B, dispatch):
     """The fused append on the single-wave kernel: the pool after the call
@@ -150,6 +155,9 @@ def test_fused_append_single_wave(dt, mode, D, B, dispatch):
     if mode == "cta":
         dispatch(pkv.DISPATCH_WAVE_CTA)
         lens, part = [1, 2, 15, 16, 17, 31, 33, 100, 511, 512, 513, 1000], 256
+    elif mode == "cta8":  # 7 x 4 KV heads x 4 partitions: one 8-warp CTA per SM at most
+        dispatch(pkv.DISPATCH_WAVE_CTA8)
+        lens, part = [1, 2, 17, 33, 511, 513, 1000], 256
     else:
         lens, part = [1, 2, 8, 9, 15, 16, 17, 31, 32, 33, 48, 63, 64], 0
     c = make_random_case("fw", 16, 4, D, B, lens, DT[dt], seed=D + B, device=DEV,
@@ -169,7 +177,8 @@ def test_fused_append_single_wave(dt, mode, D, B, dispatch):
     assert_close_to_oracle(out, ref, DT[dt], f"fused {mode} {dt} D{D} B{B}")
 
 
-@pytest.mark.parametrize("mode", [pkv.DISPATCH_WAVE_CTA, pkv.DISPATCH_WAVE_WARP])
+@pytest.mark.parametrize("mode", [pkv.DISPATCH_WAVE_CTA, pkv.DISPATCH_WAVE_CTA8,
+                                  pkv.DISPATCH_WAVE_WARP])
 @pytest.mark.parametrize("B,entry", [(16, 1), (8, 1), (8, 2)])
 def test_bad_block_id_reports_and_masks(mode, B, entry, dispatch):
     dispatch(mode)
@@ -186,7 +195,8 @@ def test_bad_block_id_reports_and_masks(mode, B, entry, dispatch):
     assert not torch.isnan(got).any()
 
 
-@pytest.mark.parametrize("mode", [pkv.DISPATCH_WAVE_CTA, pkv.DISPATCH_WAVE_WARP])
+@pytest.mark.parametrize("mode", [pkv.DISPATCH_WAVE_CTA, pkv.DISPATCH_WAVE_CTA8,
+                                  pkv.DISPATCH_WAVE_WARP])
 def test_context_len_above_max_reports(mode, dispatch):
     dispatch(mode)
     c = make_random_case("clamp_w", 8, 2, 64, 16, [30, 50], torch.float16, seed=2, device=DEV)
