@@ -124,14 +124,19 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  *     head) form a thread-block cluster (at most 16) whose first CTA merges
  *     them through distributed shared memory. Contexts of at most 64 tokens
  *     are attended one warp per (sequence, KV head). The workspace is not
- *     touched (it is still validated), and shared-prefix grouping does not
- *     apply. Under PKV_PARTITION_AUTO this kernel chooses its own partition
+ *     touched (it is still validated) except by the split form below, and
+ *     shared-prefix grouping does not apply. Under PKV_PARTITION_AUTO this kernel chooses its own partition
  *     length: the most partitions (of at least 64 tokens, at most 16) that
  *     keep the call within one wave.
  *
  * A single-wave CTA has 4 warps, or 8 when the call has at most one CTA per
  * SM and every warp gets at least two 16-token tiles (so that each SM
- * sub-partition still runs two warps).
+ * sub-partition still runs two warps). Under PKV_PARTITION_AUTO, a few very
+ * long contexts (tens of thousands of tokens on a handful of (sequence, KV
+ * head) pairs) are spread over several clusters of 8 CTAs per pair: each
+ * cluster merges its partitions into a workspace slot, and a second launch
+ * merges the slots into out. The workspace is then used (its partition
+ * slots), as by the persistent kernel.
  *
  * PKV_DISPATCH_AUTO (the default) takes the single-wave kernel whenever the
  * call fits it, else the persistent one. PKV_DISPATCH_PERSISTENT always takes

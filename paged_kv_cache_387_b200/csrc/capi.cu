@@ -88,7 +88,8 @@ std::atomic<int> g_dispatch{PKV_DISPATCH_AUTO};
 //     it so. CTAs of 8 warps when they are at most one per SM and every warp
 //     gets at least two tiles, else 4.
 bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requested_part,
-               bool *warp_items, int *warps, int *parts, int *part_tokens) {
+               bool *warp_items, int *warps, int *parts, int *part_tokens, int *clusters) {
+  *clusters = 1;
   const int mode = g_dispatch.load(std::memory_order_relaxed);
   if (mode == PKV_DISPATCH_PERSISTENT) return false;
   const long long items = (long long)a.num_seqs * a.num_kv_heads;
@@ -162,6 +163,36 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
       }
     } else if (fits8(P, pt)) {
       nw = 8;
+    }
+  }
+  // Very long contexts on few (sequence, KV head) pairs: one cluster each
+  // leaves most of the GPU idle. Several clusters of WAVE_SPLIT_CLUSTER CTAs
+  // per pair then each merge their partitions into a workspace slot, and a
+  // merge launch combines the slots. Taken when it shortens every warp's
+  // chain of tiles by WAVE_SPLIT_MIN_GAIN tiles or more (about the cost of
+  // the extra launch).
+  if (auto_part && mode == PKV_DISPATCH_AUTO && a.ws_o != nullptr) {
+    constexpr long long Pc = pkv::WAVE_SPLIT_CLUSTER;
+    int capc = 0;
+    if (pkv::decode_wave_capacity(a, dtype, false, 4, (int)Pc, &capc) == cudaSuccess &&
+        items > 0) {
+      long long C = capc / items;
+      if (C > a.max_parts) C = a.max_parts;  // workspace slots
+      for (; C >= 2; --C) {
+        long long pt2 = ((max_len + C * Pc - 1) / (C * Pc) + 15) / 16 * 16;
+        if (pt2 < 16 * pkv::WAVE_MIN_PART_TILES) pt2 = 16 * pkv::WAVE_MIN_PART_TILES;
+        const long long C2 = (parts_of(pt2) + Pc - 1) / Pc;
+        const long long chain1 = (pt / 16 + nw - 1) / nw;  // tiles per warp, one level
+        const long long chain2 = (pt2 / 16 + 3) / 4;
+        if (C2 >= 2 && C2 <= C && chain1 - chain2 >= pkv::WAVE_SPLIT_MIN_GAIN) {
+          *warp_items = false;
+          *warps = 4;
+          *parts = (int)Pc;
+          *part_tokens = (int)pt2;
+          *clusters = (int)C2;
+          return true;
+        }
+      }
     }
   }
   *warp_items = false;
@@ -352,13 +383,17 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
       return PKV_ECUDA;
     // A call that fits one wave of CTAs: one launch, no plan, no workspace.
     bool warp_items = false;
-    int wwarps = 4, wparts = 1, wtokens = 0;
-    if (plan_wave(a, dtype, auto_part, requested_part, &warp_items, &wwarps, &wparts, &wtokens)) {
-      pkv::DecodeArgs b = a;
+    int wwarps = 4, wparts = 1, wtokens = 0, wclusters = 1;
+    if (plan_wave(a, dtype, auto_part, requested_part, &warp_items, &wwarps, &wparts, &wtokens,
+                  &wclusters)) {
+      pkv::DecodeArgs b = a;  // (max_parts stays the workspace's slot stride)
       b.part_tokens = wtokens;
-      b.max_parts = wparts;
-      return cuda_status(
-          pkv::launch_decode_wave(b, dtype, warp_items, wwarps, wparts, tmK, tmV, st));
+      b.wave_clusters = wclusters;
+      e = pkv::launch_decode_wave(b, dtype, warp_items, wwarps, wparts, tmK, tmV, st);
+      if (e != cudaSuccess || wclusters <= 1) return cuda_status(e);
+      // combine the clusters' slots: a slot spans wparts partitions
+      b.part_tokens = wtokens * wparts;
+      return cuda_status(pkv::launch_merge(b, dtype, st));
     }
     // plan + decode; the partition merge is fused into the decode kernel
     return cuda_status(pkv::launch_decode_tc(a, dtype, tmK, tmV, st));

@@ -139,6 +139,9 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const DecodeArgs a
   constexpr int R = MERGE_THREADS / V;   // partition rows read concurrently
   __shared__ float scratch[MERGE_THREADS / 32];
   __shared__ float4 red[MERGE_THREADS];
+  // A programmatic dependent of the decode grid that wrote the partials (a
+  // plain stream-ordered launch otherwise): wait for it to complete.
+  pdl_wait();
 
   const int hq = blockIdx.x;
   const int s = blockIdx.y;
@@ -195,9 +198,16 @@ __global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(const DecodeArgs a
 
 template <typename T, int D>
 cudaError_t launch_merge_t(const DecodeArgs &a, cudaStream_t stream) {
-  dim3 grid(a.num_heads, a.num_seqs);
-  merge_kernel<T, D><<<grid, MERGE_THREADS, 0, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.num_heads, a.num_seqs);
+  cfg.blockDim = dim3(MERGE_THREADS);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel<T, D>, a);
 }
 
 }  // namespace

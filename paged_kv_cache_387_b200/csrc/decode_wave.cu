@@ -132,9 +132,12 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
     h = active ? (int)(item - (long long)s * Hkv) : 0;
     p = 0;
   } else {
-    p = blockIdx.x;
+    // blockIdx.z = s * C + c: cluster c of sequence s's KV head h holds
+    // partitions c * P .. c * P + P - 1, one per CTA (rank blockIdx.x).
+    const int C = max(1, a.wave_clusters);
     h = blockIdx.y;
-    s = blockIdx.z;
+    s = blockIdx.z / C;
+    p = (blockIdx.z - s * C) * gridDim.x + blockIdx.x;
     active = !stale;
   }
   const int raw_len = active ? __ldg(a.context_lens + s) : 0;
@@ -485,7 +488,15 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
 
     if (gridDim.x > 1) {  // a cluster of the P partitions (uniform over the cluster)
       cluster_sync_all();  // every partition's result is in its CTA's shared memory
-      if (active && p == 0 && nparts > 1) {  // (uniform over the CTA)
+      // This cluster's partitions q0 .. q0 + cnt - 1 of the sequence's nparts.
+      // With at most one cluster's worth, rank 0 writes the output; otherwise
+      // it writes the cluster's result (normalised o, log2-sum-exp) to
+      // workspace slot q0 / P, for the merge launch that follows.
+      const int P = gridDim.x;
+      const int q0 = p - blockIdx.x;
+      const int cnt = min(P, nparts - q0);
+      const bool to_out = nparts <= P;
+      if (active && blockIdx.x == 0 && nparts > 1 && cnt >= 1) {  // (uniform over the CTA)
         float *const wts = sc;  // [8][WAVE_MAX_PARTS] partition weights (scales are done)
         if (threadIdx.x < G) {
           const int n = threadIdx.x;
@@ -494,7 +505,7 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
           float M = -INFINITY;
 #pragma unroll
           for (int q = 0; q < WAVE_MAX_PARTS; ++q) {
-            lq[q] = q < nparts ? ld_cluster_f32(cluster_map(lse_addr, q)) : -INFINITY;
+            lq[q] = q < cnt ? ld_cluster_f32(cluster_map(lse_addr, q)) : -INFINITY;
             M = fmaxf(M, lq[q]);
           }
           float W = 0.f;
@@ -506,6 +517,9 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
           const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
           for (int q = 0; q < WAVE_MAX_PARTS; ++q) wts[n * WAVE_MAX_PARTS + q] = lq[q] * inv;
+          if (!to_out)
+            a.ws_lse[((size_t)s * Hq + h * G + n) * a.max_parts + q0 / P] =
+                W > 0.f ? M + lg2_approx(W) : -INFINITY;
         }
         __syncthreads();
         T *const out = static_cast<T *>(a.out) + ((size_t)s * Hq + h * G) * D;
@@ -513,7 +527,7 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
         for (int idx = threadIdx.x * 4; idx < G * D; idx += WV_THREADS * 4) {
           const int n = idx / D;
           float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < nparts; ++q) {
+          for (int q = 0; q < cnt; ++q) {
             const float w = wts[n * WAVE_MAX_PARTS + q];
             const float4 v = ld_cluster_f32x4(cluster_map(po + idx * 4, q));
             o.x += w * v.x;
@@ -521,10 +535,16 @@ __global__ void __launch_bounds__(NW * 32, 8 / NW)
             o.z += w * v.z;
             o.w += w * v.w;
           }
-          uint2 packed;
-          packed.x = pack2<T>(o.x, o.y);
-          packed.y = pack2<T>(o.z, o.w);
-          *reinterpret_cast<uint2 *>(out + idx) = packed;
+          if (to_out) {
+            uint2 packed;
+            packed.x = pack2<T>(o.x, o.y);
+            packed.y = pack2<T>(o.z, o.w);
+            *reinterpret_cast<uint2 *>(out + idx) = packed;
+          } else {
+            const size_t row = (size_t)s * Hq + h * G + n;
+            *reinterpret_cast<float4 *>(a.ws_o + (row * a.max_parts + q0 / P) * D + (idx - n * D)) =
+                o;
+          }
         }
       }
       cluster_sync_all();  // rank 0 has finished reading its peers' shared memory
@@ -611,7 +631,8 @@ cudaError_t launch_wave_t(const DecodeArgs &a, int parts, const CUtensorMap &tmK
     const long long items = (long long)a.num_seqs * a.num_kv_heads;
     cfg.gridDim = dim3((unsigned)((items + NW - 1) / NW));
   } else {
-    cfg.gridDim = dim3((unsigned)parts, (unsigned)a.num_kv_heads, (unsigned)a.num_seqs);
+    cfg.gridDim = dim3((unsigned)parts, (unsigned)a.num_kv_heads,
+                       (unsigned)(a.num_seqs * max(1, a.wave_clusters)));
   }
   cfg.blockDim = dim3(Shape::THREADS);
   cfg.dynamicSmemBytes = Shape::SMEM_BYTES;

@@ -52,6 +52,8 @@ struct DecodeArgs {
   int32_t *grp_tiles;  // [S] a leader's group tiles: shared + every member's own
   int unit8;           // 1 when block_size % 16 == 8: a 16-token tile is two 8-token units
                        // that may sit in different blocks
+  int wave_clusters;   // single-wave kernel: clusters per (sequence, KV head); above 1 each
+                       // writes its merged partitions to a workspace slot (0 or 1: one)
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
@@ -64,6 +66,11 @@ constexpr int WAVE_WARP_TILES = 4;
 // Under PKV_PARTITION_AUTO a single-wave partition holds at least this many
 // tiles (one per warp).
 constexpr int WAVE_MIN_PART_TILES = 4;
+// Very long contexts: clusters of this many CTAs, several per (sequence, KV
+// head), when that shortens each warp's chain of tiles by at least
+// WAVE_SPLIT_MIN_GAIN tiles.
+constexpr int WAVE_SPLIT_CLUSTER = 8;
+constexpr int WAVE_SPLIT_MIN_GAIN = 16;
 
 // Decode workspace, in order: scheduling words (256 B), the work list, the
 // per-sequence group words (two int32 per sequence), then

@@ -243,3 +243,32 @@ def test_back_to_back_single_wave_calls_in_a_graph():
         torch.cuda.synchronize()
         for o in outs:
             assert torch.equal(o, ref)
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+@pytest.mark.parametrize("lens,fused", [([65536], False), ([65536], True), ([100000], False),
+                                        ([131072], False)])
+def test_long_contexts_split_over_clusters(dt, lens, fused):
+    """A few very long contexts under PARTITION_AUTO: several clusters per
+    (sequence, KV head) each merge their partitions into a workspace slot,
+    and a merge launch combines the slots. The plan's words at the start of
+    the workspace stay untouched (no persistent kernel ran); the slots do not."""
+    c = make_random_case("split_w", 32, 8, 128, 16, lens, DT[dt], seed=len(lens) + lens[0] % 7,
+                         device=DEV, with_append=fused)
+    ws = ws_for(c, pkv.PARTITION_AUTO)
+    err = new_err(DEV)
+    if fused:
+        kc, vc = c.k_pool.cpu(), c.v_pool.cpu()
+        oracle.cache_append(kc, vc, c.k_new.cpu(), c.v_new.cpu(), c.slot_mapping.cpu())
+        ref = oracle.paged_decode(c.q.cpu(), kc, vc, c.block_tables.cpu(), c.context_lens.cpu(),
+                                  c.scale)
+    else:
+        ref = oracle_decode(c)
+    got = decode_ws(c, pkv.PARTITION_AUTO, ws, err=err, fused=fused)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert (ws[:256] == 0xAB).all()
+    assert not (ws == 0xAB).all()
+    if fused:
+        assert torch.equal(c.k_pool.cpu().view(torch.int16), kc.view(torch.int16))
+    assert_close_to_oracle(got, ref, DT[dt], f"split clusters {dt} {lens}")
