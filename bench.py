@@ -544,8 +544,9 @@ def time_fused_call(pkv, case, steps, warmup, stream):
 
 # Small calls: Llama-8B heads (32 query / 8 KV, d128), bf16, 16-token blocks,
 # one step of the fused append + decode with PARTITION_AUTO.
-SMALL_BATCHES = {"1x16": [16], "1x4096": [4096], "1x8192": [8192], "4x16384": [16384] * 4,
-                 "32x1024": [1024] * 32, "256x16": [16] * 256}
+SMALL_BATCHES = {"1x16": [16], "1x4096": [4096], "1x8192": [8192], "1x32768": [32768],
+                 "1x131072": [131072], "4x16384": [16384] * 4, "32x1024": [1024] * 32,
+                 "256x16": [16] * 256}
 
 
 def small_batch_lines(pkv, dev, stream, shapes=None):
@@ -553,7 +554,7 @@ def small_batch_lines(pkv, dev, stream, shapes=None):
     (these calls take the single-wave kernel) and with the persistent kernel
     forced:
       graph_us: 50 back-to-back calls replayed from a CUDA graph, per call
-        (the K/V, 0.5-134 MB, stays in the 126 MB L2 when it fits);
+        (the K/V, 0.07-537 MB, stays in the 126 MB L2 when it fits);
       cold_us: one call after a 256 MB write has evicted L2, timed by events
         around it (median of 15), with its K/V GB/s."""
     import torch
