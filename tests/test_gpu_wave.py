@@ -272,3 +272,25 @@ def test_long_contexts_split_over_clusters(dt, lens, fused):
     if fused:
         assert torch.equal(c.k_pool.cpu().view(torch.int16), kc.view(torch.int16))
     assert_close_to_oracle(got, ref, DT[dt], f"split clusters {dt} {lens}")
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,B,dt", [(8, 1, 64, 8, "f16"), (16, 2, 128, 32, "bf16"),
+                                           (6, 2, 64, 16, "bf16")])
+def test_split_form_shapes(Hq, Hkv, D, B, dt):
+    """The split form over head dims, block sizes (8: two blocks per tile) and
+    group sizes, with up to 32 clusters per KV head; fused append included."""
+    c = make_random_case("split_shapes", Hq, Hkv, D, B, [65536], DT[dt], seed=Hq + D + B,
+                         device=DEV, with_append=True)
+    kc, vc = c.k_pool.cpu(), c.v_pool.cpu()
+    oracle.cache_append(kc, vc, c.k_new.cpu(), c.v_new.cpu(), c.slot_mapping.cpu())
+    ref = oracle.paged_decode(c.q.cpu(), kc, vc, c.block_tables.cpu(), c.context_lens.cpu(),
+                              c.scale)
+    ws = ws_for(c, pkv.PARTITION_AUTO)
+    err = new_err(DEV)
+    got = decode_ws(c, pkv.PARTITION_AUTO, ws, err=err, fused=True)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert (ws[:256] == 0xAB).all()
+    assert not (ws == 0xAB).all()
+    assert torch.equal(c.v_pool.cpu().view(torch.int16), vc.view(torch.int16))
+    assert_close_to_oracle(got, ref, DT[dt], f"split D{D} B{B} G{Hq // Hkv}")
