@@ -31,9 +31,10 @@
 //   most two descriptors, which spreads the final items over the CTAs. It
 //   also keeps the partition count. When the consumers finish an item of a
 //   split context, the scheduler publishes it (a device-scope fence and a
-//   fetch-and-add on the (sequence, KV head) counter). The CTA that completes
-//   the last partition receives a merge task in its descriptor stream. No CTA
-//   ever waits for another.
+//   fetch-and-add on its chunk's counter). The scheduler warp that completes a
+//   chunk of 16 partitions merges it right away, and the one that completes
+//   the last chunk merges the chunks into `out`: the merges never queue behind
+//   work items in a descriptor ring. No CTA ever waits for another.
 //   Warps 0-3 are consumers. Each owns a ring of stages in shared memory and
 //   takes tiles w, w+4, w+8, ... of every item. Its lane 0 fills the ring
 //   with TMA, completing on the stage's mbarrier:
@@ -100,10 +101,8 @@ constexpr float RESCALE_SLACK = 8.f;     // lazy max: rescale only past 2^8 grow
 
 // Descriptor kinds (in ItemDesc::kind).
 constexpr int KIND_WORK = 0;         // attend one (sequence, partition, KV head)
-constexpr int KIND_MERGE_CHUNK = 1;  // merge partitions of chunk p into a chunk result
-constexpr int KIND_MERGE_FINAL = 2;  // merge partitions (one chunk) or chunk results into out
-constexpr int KIND_NOP = 3;          // keeps the ring turning while the last items finish
-constexpr int KIND_END = 4;          // no more descriptors
+constexpr int KIND_NOP = 1;          // keeps the ring turning while the last items finish
+constexpr int KIND_END = 2;          // no more descriptors
 constexpr int PLAN_BUCKETS = 64;     // size classes for ordering the short last partitions
 
 // Most sequences one work item attends together (a shared-prefix group).
@@ -734,38 +733,44 @@ __device__ __forceinline__ bool consumers_all(bool v) {
 // o = sum_q 2^(lse_q - lse) o_q with lse = log2 sum_q 2^lse_q. The sources
 // were written by other CTAs; they are read from L2 (ld.global.cg). The
 // result goes to `out` (final), or to chunk entry `dst_idx` of the
-// second-level arrays as (o, lse).
+// second-level arrays as (o, lse). Threads tid = 0 .. nthreads-1 share it.
 template <typename T, int D>
 __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int G, int members,
                                          const float *src_o, const float *src_lse,
                                          int src_stride, int q0, int q1, bool final_out,
-                                         int dst_idx) {
+                                         int dst_idx, int tid, int nthreads) {
   constexpr int V = D / 4;  // float4 columns per head row
   T *const out = static_cast<T *>(a.out);
   const int n_q = q1 - q0;
-  for (int idx = threadIdx.x; idx < members * G * V; idx += NCW * 32) {
+  for (int idx = tid; idx < members * G * V; idx += nthreads) {
     const int n = idx / V;
     const int cv = idx - n * V;
     const int mem = n / G;
     const size_t row = (size_t)(s + mem) * a.num_heads + h * G + (n - mem * G);
     const float *lse = src_lse + row * src_stride + q0;
     const float4 *po = reinterpret_cast<const float4 *>(src_o + (row * src_stride + q0) * D) + cv;
+    // All of the entries' loads are issued before the first is used.
+    float lq[MERGE_CHUNK];
+    float4 vq[MERGE_CHUNK];
+#pragma unroll
+    for (int q = 0; q < MERGE_CHUNK; ++q) {
+      lq[q] = q < n_q ? __ldcg(lse + q) : -INFINITY;
+      vq[q] = q < n_q ? __ldcg(po + (size_t)q * V) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float M = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < MERGE_CHUNK; ++q)
-      if (q < n_q) M = fmaxf(M, __ldcg(lse + q));
+    for (int q = 0; q < MERGE_CHUNK; ++q) M = fmaxf(M, lq[q]);
     float W = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (M != -INFINITY) {
-#pragma unroll 4
-      for (int q = 0; q < n_q; ++q) {
-        const float w = exp2f(__ldcg(lse + q) - M);
-        const float4 v = __ldcg(po + (size_t)q * V);
+#pragma unroll
+      for (int q = 0; q < MERGE_CHUNK; ++q) {
+        const float w = lq[q] == -INFINITY ? 0.f : exp2f(lq[q] - M);
         W += w;
-        acc.x += w * v.x;
-        acc.y += w * v.y;
-        acc.z += w * v.z;
-        acc.w += w * v.w;
+        acc.x += w * vq[q].x;
+        acc.y += w * vq[q].y;
+        acc.z += w * vq[q].z;
+        acc.w += w * vq[q].w;
       }
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
@@ -783,6 +788,12 @@ __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int 
       if (cv == 0) a.ws2_lse[row * a.max_chunks + dst_idx] = W > 0.f ? M + log2f(W) : -INFINITY;
     }
   }
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // Where group tile gt of a work item lies: in the shared span (m = -1; every
@@ -884,64 +895,64 @@ __global__ void __launch_bounds__(THREADS, 2)
     bool first_post = true;
     int item = blockIdx.x;  // the counter starts at grid
     bool claimed = true;  // `item` holds an index taken from the work list
-    int in_flight = 0;    // posted work / merge descriptors whose completion is not yet handled
+    int in_flight = 0;    // posted work descriptors whose completion is not yet handled
     uint32_t it = 0;      // descriptors posted
     for (;; ++it) {
       const int slot = it % NSLOT;
       ItemDesc &d = desc[slot];
-      int merge_kind = -1, merge_s = 0, merge_h = 0, merge_np = 0, merge_p = 0, merge_m = 1;
       if (it >= NSLOT) {
         if (!__all_sync(FULL_MASK, wait_or_abort(item_empty(slot), ((it / NSLOT) - 1) & 1,
                                                  abort_flag, a.err)))
           break;
-        // The consumers are done with the slot's previous descriptor: publish
-        // a finished partition / chunk result and post the merge it completes.
+        // The consumers are done with the slot's previous descriptor. A
+        // finished partition of a split context is published (a device-scope
+        // fence, then a fetch-and-add on its chunk's counter); the warp that
+        // completes a chunk merges it here at once, and the one that completes
+        // the last chunk merges the chunks into `out`. Merging here, not in
+        // the consumers' descriptor stream, keeps the merges from queueing
+        // behind the work items already posted.
         const int pk = d.kind;
-        if (pk == KIND_WORK || pk == KIND_MERGE_CHUNK || pk == KIND_MERGE_FINAL) --in_flight;
+        if (pk == KIND_WORK) --in_flight;
         const int np = d.nparts;
-        const int nchunks = (np + MERGE_CHUNK - 1) / MERGE_CHUNK;
-        int next_kind = -1, next_p = 0;
-        if (lane == 0 && ((pk == KIND_WORK && np > 1) || pk == KIND_MERGE_CHUNK)) {
-          __threadfence();
-          if (pk == KIND_WORK) {
-            const int ch = d.p / MERGE_CHUNK;
-            const int ch_size = min(MERGE_CHUNK, np - ch * MERGE_CHUNK);
-            const int t = atomicAdd(&a.merge_cnt[(d.s * Hkv + d.h) * a.max_chunks + ch], 1);
-            if (t == ch_size - 1) {
-              next_kind = nchunks == 1 ? KIND_MERGE_FINAL : KIND_MERGE_CHUNK;
-              next_p = ch;
-            }
-          } else {
-            const int t = atomicAdd(&a.merge_cnt2[d.s * Hkv + d.h], 1);
-            if (t == nchunks - 1) next_kind = KIND_MERGE_FINAL;
+        if (pk == KIND_WORK && np > 1) {
+          const int ms = d.s, mh = d.h, mm = d.members, ch = d.p / MERGE_CHUNK;
+          const int nchunks = (np + MERGE_CHUNK - 1) / MERGE_CHUNK;
+          int32_t *const cnt1 = &a.merge_cnt[(ms * Hkv + mh) * a.max_chunks + ch];
+          int32_t *const cnt2 = &a.merge_cnt2[ms * Hkv + mh];
+          int t = 0;
+          if (lane == 0) {
+            __threadfence();
+            t = atomicAdd(cnt1, 1);
           }
-          if (next_kind >= 0) __threadfence();
-        }
-        next_kind = __shfl_sync(FULL_MASK, next_kind, 0);
-        if (next_kind >= 0) {
-          merge_kind = next_kind;
-          merge_s = d.s;
-          merge_h = d.h;
-          merge_np = np;
-          merge_m = d.members;
-          merge_p = __shfl_sync(FULL_MASK, next_p, 0);
+          const int ch_size = min(MERGE_CHUNK, np - ch * MERGE_CHUNK);
+          if (__shfl_sync(FULL_MASK, t, 0) == ch_size - 1) {
+            (void)ld_acquire_gpu(cnt1);  // every lane: the chunk's partials are visible
+            bool final_ready = nchunks == 1;
+            if (!final_ready) {
+              merge_range<T, D>(a, ms, mh, G, mm, a.ws_o, a.ws_lse, a.max_parts,
+                                ch * MERGE_CHUNK, ch * MERGE_CHUNK + ch_size, false, ch, lane, 32);
+              __threadfence();  // every lane's chunk result precedes the count
+              __syncwarp();
+              int t2 = 0;
+              if (lane == 0) {
+                __threadfence();
+                t2 = atomicAdd(cnt2, 1);
+              }
+              final_ready = __shfl_sync(FULL_MASK, t2, 0) == nchunks - 1;
+              if (final_ready) (void)ld_acquire_gpu(cnt2);  // the other chunks' results
+            }
+            if (final_ready) {
+              if (nchunks == 1)
+                merge_range<T, D>(a, ms, mh, G, mm, a.ws_o, a.ws_lse, a.max_parts, 0, np, true,
+                                  0, lane, 32);
+              else
+                merge_range<T, D>(a, ms, mh, G, mm, a.ws2_o, a.ws2_lse, a.max_chunks, 0, nchunks,
+                                  true, 0, lane, 32);
+            }
+          }
         }
       }
       __syncwarp();  // every lane has read the old descriptor before it is rewritten
-      if (merge_kind >= 0) {
-        if (lane == 0) {
-          d.kind = merge_kind;
-          d.s = merge_s;
-          d.h = merge_h;
-          d.p = merge_p;
-          d.nparts = merge_np;
-          d.members = merge_m;
-          d.n_tiles = 0;
-          mbar_arrive(item_full(slot));
-        }
-        ++in_flight;
-        continue;
-      }
       if (!claimed) {
         // End phase: claim the next item only once the descriptor posted two
         // iterations ago is done, so at most two work descriptors are held.
@@ -957,7 +968,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       if (item >= total_items) {
         // No new work: keep the ring turning (no-op descriptors) until every
-        // posted item has completed and produced its merge tasks, then stop.
+        // posted item has completed (and its merges are done), then stop.
         if (lane == 0) {
           d.kind = in_flight == 0 ? KIND_END : KIND_NOP;
           d.n_tiles = 0;
@@ -1255,20 +1266,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const ItemDesc &dref = desc[slot];
     const int kind = dref.kind;
     if (kind == KIND_END) break;  // the same descriptor for every consumer: a uniform exit
-    if (kind != KIND_WORK) {
-      const int np = dref.nparts;
-      if (kind == KIND_MERGE_CHUNK) {
-        const int q0 = dref.p * MERGE_CHUNK;
-        merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws_o, a.ws_lse, a.max_parts, q0,
-                          min(np, q0 + MERGE_CHUNK), false, dref.p);
-      } else if (kind == KIND_MERGE_FINAL) {
-        if (np <= MERGE_CHUNK)
-          merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws_o, a.ws_lse, a.max_parts,
-                            0, np, true, 0);
-        else
-          merge_range<T, D>(a, dref.s, dref.h, G, dref.members, a.ws2_o, a.ws2_lse,
-                            a.max_chunks, 0, (np + MERGE_CHUNK - 1) / MERGE_CHUNK, true, 0);
-      }
+    if (kind != KIND_WORK) {  // a no-op that keeps the ring turning
       pump(false);
       consumers_sync();  // the descriptor is read by all before the slot is handed back
       if (lane == 0) mbar_arrive(item_empty(slot));
