@@ -139,7 +139,10 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  * slots), as by the persistent kernel.
  *
  * PKV_DISPATCH_AUTO (the default) takes the single-wave kernel whenever the
- * call fits it, else the persistent one. PKV_DISPATCH_PERSISTENT always takes
+ * call fits it and no warp gets more than 64 16-token tiles, else the
+ * persistent one. (The single-wave kernel fixes one CTA per partition. Only
+ * max_context_len is known on the host, so one long sequence among short ones
+ * would run on a few CTAs there, while the persistent kernel spreads it.) PKV_DISPATCH_PERSISTENT always takes
  * the persistent kernel. PKV_DISPATCH_WAVE_CTA never uses the warp-per-item
  * form and keeps CTAs at 4 warps; PKV_DISPATCH_WAVE_CTA8 never uses the
  * warp-per-item form and takes 8-warp CTAs whenever they fit one per SM.

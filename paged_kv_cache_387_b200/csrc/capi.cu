@@ -184,7 +184,8 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
         const long long C2 = (parts_of(pt2) + Pc - 1) / Pc;
         const long long chain1 = (pt / 16 + nw - 1) / nw;  // tiles per warp, one level
         const long long chain2 = (pt2 / 16 + 3) / 4;
-        if (C2 >= 2 && C2 <= C && chain1 - chain2 >= pkv::WAVE_SPLIT_MIN_GAIN) {
+        if (C2 >= 2 && C2 <= C && chain1 - chain2 >= pkv::WAVE_SPLIT_MIN_GAIN &&
+            (mode != PKV_DISPATCH_AUTO || chain2 <= pkv::WAVE_MAX_WARP_CHAIN)) {
           *warp_items = false;
           *warps = 4;
           *parts = (int)Pc;
@@ -195,6 +196,12 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
       }
     }
   }
+  // One CTA per partition, with no balancing between them: under the default
+  // selection a partition may not give a warp more than WAVE_MAX_WARP_CHAIN
+  // tiles, or one long sequence among short ones would run on few CTAs while
+  // the persistent kernel spreads it.
+  if (mode == PKV_DISPATCH_AUTO && (pt / 16 + nw - 1) / nw > pkv::WAVE_MAX_WARP_CHAIN)
+    return false;
   *warp_items = false;
   *warps = nw;
   *parts = (int)P;

@@ -71,6 +71,10 @@ constexpr int WAVE_MIN_PART_TILES = 4;
 // WAVE_SPLIT_MIN_GAIN tiles.
 constexpr int WAVE_SPLIT_CLUSTER = 8;
 constexpr int WAVE_SPLIT_MIN_GAIN = 16;
+// Under the default selection, the single-wave kernel takes a call only if no
+// warp gets more than this many 16-token tiles (its partitions are fixed per
+// CTA; the persistent kernel balances ragged lengths instead).
+constexpr int WAVE_MAX_WARP_CHAIN = 64;
 
 // Decode workspace, in order: scheduling words (256 B), the work list, the
 // per-sequence group words (two int32 per sequence), then
