@@ -80,13 +80,18 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ECUDA; }
 std::atomic<int> g_dispatch{PKV_DISPATCH_AUTO};
 
 // Launch shape of a single-wave decode for a 16-bit call, or false when the
-// call does not fit one wave of CTAs (the persistent kernel takes it then).
+// persistent kernel takes the call.
 //   warp mode: every context fits WAVE_WARP_TILES tiles and one partition;
 //   CTA mode: S * Hkv * P CTAs (P partitions of part_tokens each, P <=
 //     WAVE_MAX_PARTS) are resident at once. Under PKV_PARTITION_AUTO, P is
 //     the most partitions (of at least WAVE_MIN_PART_TILES tiles) that keep
 //     it so. CTAs of 8 warps when they are at most one per SM and every warp
-//     gets at least two tiles, else 4.
+//     gets at least two tiles, else 4;
+//   split form (PKV_PARTITION_AUTO, very long contexts): `clusters` clusters
+//     of WAVE_SPLIT_CLUSTER CTAs per (sequence, KV head), merged afterwards
+//     through the workspace.
+// Under the default selection no warp may get more than WAVE_MAX_WARP_CHAIN
+// tiles.
 bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requested_part,
                bool *warp_items, int *warps, int *parts, int *part_tokens, int *clusters) {
   *clusters = 1;
@@ -185,7 +190,7 @@ bool plan_wave(const pkv::DecodeArgs &a, int dtype, bool auto_part, int requeste
         const long long chain1 = (pt / 16 + nw - 1) / nw;  // tiles per warp, one level
         const long long chain2 = (pt2 / 16 + 3) / 4;
         if (C2 >= 2 && C2 <= C && chain1 - chain2 >= pkv::WAVE_SPLIT_MIN_GAIN &&
-            (mode != PKV_DISPATCH_AUTO || chain2 <= pkv::WAVE_MAX_WARP_CHAIN)) {
+            chain2 <= pkv::WAVE_MAX_WARP_CHAIN) {
           *warp_items = false;
           *warps = 4;
           *parts = (int)Pc;
