@@ -66,6 +66,10 @@ def parse_args():
                          "the first upload and the last download, which nothing overlaps")
     ap.add_argument("--e2e-buffers", type=int, default=4,
                     help="device input/output buffers in the end-to-end loop (>= 2)")
+    ap.add_argument("--e2e-steps-per-upload", type=int, default=4,
+                    help="end-to-end loop: steps whose inputs go up in one copy and whose "
+                         "results come back in one copy (>= 1); the calls of a group run "
+                         "back to back on the compute stream")
     ap.add_argument("--e2e-compute-streams", type=int, default=1,
                     help="compute streams that take turns with the end-to-end loop's steps, "
                          "each with its own workspace (>= 1)")
@@ -761,10 +765,12 @@ def run_ours(args, rank, world, local_rank):
     value = whole_job_gbs(dec_bytes + app_bytes, world, ms * 1e-3)
 
     # ---- end to end: host buffers, copies inside the timed region ----
-    # Every step uploads its own inputs from pinned host memory and gets its
-    # result back to the host, as a serving loop does. Uploads and downloads
-    # run on two copy streams with `--e2e-buffers` device buffers, so later
-    # steps' uploads and earlier steps' downloads overlap a step's kernels.
+    # Every step's inputs go up from pinned host memory and every step's
+    # result comes back to the host, as in a serving loop; the inputs of
+    # `--e2e-steps-per-upload` steps travel in one copy. Uploads and
+    # downloads run on two copy streams with `--e2e-buffers` device buffers,
+    # so later groups' uploads and earlier groups' downloads overlap a
+    # group's kernels.
     # With `--e2e-result-in-host-memory` the decode writes its result straight
     # into a pinned host buffer instead (the C ABI accepts page-locked host
     # memory for `out`), leaving the copy engines to the uploads. The host
@@ -785,30 +791,12 @@ def run_ours(args, rank, world, local_rank):
 
     def views(buf):
         return {k: buf[o:o + n].view(dt).view(shp) for k, (o, n, dt, shp) in segs.items()}
-    host_stage = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
-    for k, t in views(host_stage).items():
-        t.copy_(getattr(case, k).cpu())
     nb = max(2, args.e2e_buffers)
-    dev_stage = [torch.empty(h2d, dtype=torch.uint8, device=dev) for _ in range(nb)]
-    dev_sets = [views(b) for b in dev_stage]
-    outs = [torch.empty_like(out) for _ in range(nb)]
-    host_outs = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(nb)]
-    d2h = host_outs[0].numel() * host_outs[0].element_size()
+    d2h = out.numel() * out.element_size()
     h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    # Per buffer b: in_ready (upload done), done (decode done), out_free
-    # (download done, which follows `done`). The upload into buffer b waits
-    # for out_free of the step that used b before, so a compute stream only
-    # waits for in_ready and records done. The steps take turns on
-    # `--e2e-compute-streams` compute streams, each with its own workspace:
-    # a stream operation between two calls on one stream ends the
-    # programmatic overlap of their launches, and with two streams the next
-    # step's kernels still start while the previous step's drain.
     ncs = max(1, args.e2e_compute_streams)
     comp = [stream] + [torch.cuda.Stream(dev) for _ in range(ncs - 1)]
     wss = [ws] + [torch.empty_like(ws) for _ in range(ncs - 1)]
-    in_ready = [torch.cuda.Event() for _ in range(nb)]
-    done = [torch.cuda.Event() for _ in range(nb)]
-    out_free = [torch.cuda.Event() for _ in range(nb)]
 
     def run_step(inp, o, cs, wsi):
         if fused:
@@ -824,40 +812,89 @@ def run_ours(args, rank, world, local_rank):
                               partition_size=case.partition_size, workspace=wsi, err=err,
                               stream=cs)
 
-    def e2e_steps(n, start_event=None):
-        for i in range(n):
-            b = i % nb
-            with torch.cuda.stream(h2d_stream):
-                if i >= nb:
-                    h2d_stream.wait_event(out_free[b])  # buffer b's previous step is over
-                elif start_event is not None:
-                    h2d_stream.wait_event(start_event)
-                dev_stage[b].copy_(host_stage, non_blocking=True)
-                in_ready[b].record(h2d_stream)
-            cs, wsi = comp[i % ncs], wss[i % ncs]
-            cs.wait_event(in_ready[b])
-            if args.e2e_result_in_host_memory:
-                # the decode writes its result straight into pinned host memory
-                run_step(dev_sets[b], host_outs[b], cs, wsi)
-                done[b].record(cs)
-                out_free[b] = done[b]
-                continue
-            run_step(dev_sets[b], outs[b], cs, wsi)
-            done[b].record(cs)
-            with torch.cuda.stream(d2h_stream):
-                d2h_stream.wait_event(done[b])
-                host_outs[b].copy_(outs[b], non_blocking=True)
-                out_free[b].record(d2h_stream)
-        for other in [d2h_stream] + comp[1:]:
-            last = torch.cuda.Event()
-            last.record(other)
-            stream.wait_event(last)
+    def make_e2e(G):
+        """The end-to-end loop with G steps per upload: one pinned staging
+        buffer holds G steps' inputs (each step its own segment), goes up in
+        one copy, and the G steps' results come back in one copy. Between the
+        G calls of a group no stream operation intervenes, so their launches
+        keep their programmatic overlap; every step's input and result bytes
+        still cross the host link inside the timed region."""
+        host_stage = torch.empty(G * h2d, dtype=torch.uint8, pin_memory=True)
+        for g in range(G):
+            for k, t in views(host_stage[g * h2d:(g + 1) * h2d]).items():
+                t.copy_(getattr(case, k).cpu())
+        dev_stage = [torch.empty(G * h2d, dtype=torch.uint8, device=dev) for _ in range(nb)]
+        dev_sets = [[views(b[g * h2d:(g + 1) * h2d]) for g in range(G)] for b in dev_stage]
+        outs = [torch.empty((G,) + tuple(out.shape), dtype=out.dtype, device=dev)
+                for _ in range(nb)]
+        host_outs = [torch.empty((G,) + tuple(out.shape), dtype=out.dtype, pin_memory=True)
+                     for _ in range(nb)]
+        # Per buffer b: in_ready (upload done), done (decodes done), out_free
+        # (download done, which follows `done`). The upload into buffer b
+        # waits for out_free of the group that used b before, so a compute
+        # stream only waits for in_ready and records done, once per group.
+        # Groups take turns on `--e2e-compute-streams` compute streams, each
+        # with its own workspace.
+        in_ready = [torch.cuda.Event() for _ in range(nb)]
+        done = [torch.cuda.Event() for _ in range(nb)]
+        out_free = [torch.cuda.Event() for _ in range(nb)]
 
-    e2e_steps(3)
-    torch.cuda.synchronize()
-    # The device-only step again, right before the end-to-end loop: the
+        def steps(n, start_event=None):
+            for j in range(n // G):
+                b = j % nb
+                with torch.cuda.stream(h2d_stream):
+                    if j >= nb:
+                        h2d_stream.wait_event(out_free[b])  # buffer b's previous group is over
+                    elif start_event is not None:
+                        h2d_stream.wait_event(start_event)
+                    dev_stage[b].copy_(host_stage, non_blocking=True)
+                    in_ready[b].record(h2d_stream)
+                cs, wsi = comp[j % ncs], wss[j % ncs]
+                cs.wait_event(in_ready[b])
+                if args.e2e_result_in_host_memory:
+                    # the decode writes its result straight into pinned host memory
+                    for g in range(G):
+                        run_step(dev_sets[b][g], host_outs[b][g], cs, wsi)
+                    done[b].record(cs)
+                    out_free[b] = done[b]
+                    continue
+                for g in range(G):
+                    run_step(dev_sets[b][g], outs[b][g], cs, wsi)
+                done[b].record(cs)
+                with torch.cuda.stream(d2h_stream):
+                    d2h_stream.wait_event(done[b])
+                    host_outs[b].copy_(outs[b], non_blocking=True)
+                    out_free[b].record(d2h_stream)
+            for other in [d2h_stream] + comp[1:]:
+                last = torch.cuda.Event()
+                last.record(other)
+                stream.wait_event(last)
+        return steps
+
+    def time_e2e(G):
+        steps = make_e2e(G)
+        steps(3 * G)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n = max(args.steps, args.e2e_steps) // G * G
+        e0.record(stream)
+        t0 = time.perf_counter()
+        steps(n, start_event=e0)
+        submit_ms = (time.perf_counter() - t0) * 1e3 / n
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks([e0.elapsed_time(e1) / n], dev)[0], n, submit_ms
+
+    G = max(1, args.e2e_steps_per_upload)
+    # The device-only step again, right before the end-to-end loops: the
     # ratio of the two is taken at the same clocks (the power cap moves them
     # over a run).
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_adj = min(args.steps, 100)
     a0.record(stream)
@@ -866,18 +903,9 @@ def run_ours(args, rank, world, local_rank):
     a1.record(stream)
     torch.cuda.synchronize()
     adj_ms = max_over_ranks([a0.elapsed_time(a1) / n_adj], dev)[0]
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    t_sub0 = time.perf_counter()
-    n_e2e = max(args.steps, args.e2e_steps)
-    e2e_steps(n_e2e, start_event=e0)
-    host_submit_ms = (time.perf_counter() - t_sub0) * 1e3 / n_e2e
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / n_e2e], dev)[0]
+    e2e_ms, n_e2e, host_submit_ms = time_e2e(G)
+    # the same loop with one upload and one download per step (diagnostic)
+    e2e_ms_1 = time_e2e(1)[0] if G > 1 else e2e_ms
 
     # the copy engines' own rates for this step's transfer sizes (diagnostic)
     def copy_gbs(dst, src, nbytes, reps=20):
@@ -894,7 +922,7 @@ def run_ours(args, rank, world, local_rank):
     flat_h = torch.empty(h2d, dtype=torch.uint8, pin_memory=True)
     flat_d = torch.empty(h2d, dtype=torch.uint8, device=dev)
     h2d_gbs = copy_gbs(flat_d, flat_h, h2d)
-    d2h_gbs = copy_gbs(host_outs[0], outs[0], d2h)
+    d2h_gbs = copy_gbs(torch.empty(out.shape, dtype=out.dtype, pin_memory=True), out, d2h)
     del flat_h, flat_d
     e2e_value = whole_job_gbs(dec_bytes + app_bytes, world, e2e_ms * 1e-3)
 
@@ -981,9 +1009,13 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "GB/s", "ms_per_step": e2e_ms, "steps": n_e2e,
                 "device_ms_per_step_adjacent": adj_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "pipelining": "inputs staged in one pinned buffer, one upload per step on a copy "
-                              "stream, overlapping the neighbouring steps' kernels; steps take "
-                              f"turns on {ncs} compute stream(s), each with its own workspace",
+                "steps_per_upload": G,
+                "ms_per_step_one_upload_per_step": e2e_ms_1,
+                "pipelining": f"inputs of {G} step(s) staged in one pinned buffer, one upload "
+                              "per group on a copy stream, overlapping the neighbouring groups' "
+                              "kernels; each step's result comes back in one download per "
+                              f"group; groups take turns on {ncs} compute stream(s), each with "
+                              "its own workspace",
                 "result_to_host": ("written by the decode kernels into pinned host memory"
                                    if args.e2e_result_in_host_memory else
                                    "device-to-host copy on a second copy stream"),
