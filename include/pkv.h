@@ -79,8 +79,11 @@ enum {
  * (sequence, partition) pair) and two int32 per sequence for the
  * shared-prefix grouping, plus, when a context can span several
  * partitions, merge counters and one fp32 output row and one fp32
- * log-sum-exp per (sequence, query head, partition). Always > 0 for
- * num_seqs > 0. This function is pure arithmetic: it does not touch the GPU.
+ * log-sum-exp per (sequence, query head, partition), and last the
+ * tail-split pieces: min(512, num_seqs * num_heads * partitions) of them,
+ * each a counter and 8 fp32 rows of head_dim with their log-sum-exp values
+ * (about 2 MB at head_dim 128). Always > 0 for num_seqs > 0. This function
+ * is pure arithmetic: it does not touch the GPU.
  */
 size_t pkv_decode_workspace_bytes(int num_seqs, int num_heads, int head_dim,
                                   int max_context_len, int partition_size);
@@ -117,7 +120,9 @@ int pkv_resolve_partition(int num_seqs, int num_heads, int max_context_len, int 
  *   - the persistent kernel: a one-CTA plan launch builds a work list from
  *     context_lens, then two CTAs per SM pull (sequence, partition, KV head)
  *     items, merging split contexts through the workspace. It balances large
- *     and ragged batches.
+ *     and ragged batches. With one or two query heads per KV head, when the
+ *     last items would leave more than half of the CTAs idle, each of them is
+ *     attended as up to 8 pieces and merged the same way.
  *   - the single-wave kernel: when every (sequence, KV head, partition) of
  *     the call fits in one wave of CTAs, one launch with no plan. CTA
  *     (p, h, s) attends partition p, and the partitions of one (sequence, KV

@@ -244,6 +244,14 @@ WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long lo
       off += round_up((size_t)(S * Hq * chunks) * sizeof(float), 256);
     }
   }
+  w.tail_slots = S * Hq * max_parts < pkv::TAIL_MAX_PIECES ? S * Hq * max_parts
+                                                           : pkv::TAIL_MAX_PIECES;
+  w.tcnt_off = off;
+  off += round_up((size_t)w.tail_slots * sizeof(int32_t), 256);
+  w.to_off = off;
+  off += round_up((size_t)(w.tail_slots * pkv::TAIL_COLS * D) * sizeof(float), 256);
+  w.tlse_off = off;
+  off += round_up((size_t)(w.tail_slots * pkv::TAIL_COLS) * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -369,6 +377,10 @@ int decode_impl(void *out, const void *q, const void *k_pool, const void *v_pool
   a.work = reinterpret_cast<uint2 *>(ws + wl.work_off);
   a.grp = reinterpret_cast<int32_t *>(ws + wl.grp_off);
   a.grp_tiles = a.grp + num_seqs;
+  a.tail_cnt = reinterpret_cast<int32_t *>(ws + wl.tcnt_off);
+  a.tail_o = reinterpret_cast<float *>(ws + wl.to_off);
+  a.tail_lse = reinterpret_cast<float *>(ws + wl.tlse_off);
+  a.tail_slots = (int)wl.tail_slots;
   a.max_chunks = (int)((mp + pkv::MERGE_CHUNK - 1) / pkv::MERGE_CHUNK);
   if (mp > 1) {
     a.merge_cnt = reinterpret_cast<int32_t *>(ws + wl.cnt_off);

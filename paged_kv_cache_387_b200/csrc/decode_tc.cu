@@ -19,7 +19,11 @@
 //   also resets the dispatch and merge counters. The decode kernel is
 //   persistent, two CTAs per SM. Each CTA takes item blockIdx.x first, then
 //   pulls items (pair x KV head) from an atomic counter until the list is
-//   exhausted. Launches chain by programmatic dependence: the plan is
+//   exhausted. Where the last items would leave most of the grid idle (a
+//   remainder of at most half the grid, with one or two query heads per KV
+//   head), the plan has each of them claimed as several pieces of consecutive
+//   tiles, merged like partitions (plan_tail). Launches chain by programmatic
+//   dependence: the plan is
 //   launched while the previous call finishes (and waits for it before it
 //   reads anything), and the decode grid's set-up overlaps the plan.
 //
@@ -122,6 +126,7 @@ struct alignas(16) ItemDesc {
   int own[MAX_MEMBERS + 1];  // first own tile of each member; own[members] = all tiles
   int len[MAX_MEMBERS];      // members' context lengths
   int ids[DESC_IDS];  // physical block of tile (or 8-token unit) t; -1 past the context
+  int tail;  // piece slot of a tail-split item (p = piece, nparts = pieces), or -1
 };
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base). NH is
@@ -174,6 +179,7 @@ struct TcShape {
   static_assert(NBARS <= 64, "barrier area");
   static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= CTA_SMEM_BUDGET, "two CTAs per SM");
+  static_assert(NH <= TAIL_COLS, "a tail piece slot holds every column of an item");
   static_assert(QBUF_OFF % 16 == 0 && DESC_OFF % 16 == 0 && BAR_OFF % 8 == 0, "alignment");
 };
 
@@ -390,6 +396,42 @@ __device__ __noinline__ void plan_small(const DecodeArgs &a, int lane) {
   }
 }
 
+// Tail split, decided by every thread of the plan block alike once the work
+// list (total entries, the first total_m of several partitions) is written.
+// The CTAs take items in list order, so the last wave holds the r = items mod
+// grid last items (the smallest, by the size classes) while the other CTAs
+// run out of work. When r is at most half the grid and those items are long,
+// each of them is attended as k = min(grid / r, ...) pieces of consecutive
+// tiles instead, so the last wave spreads over about r * k CTAs; the pieces'
+// partial results (in the tail region) are merged when an item's last piece
+// finishes. Only one-partition entries are split, and every piece keeps at
+// least TAIL_MIN_PIECE_TILES tiles (the last entry is the smallest). The plan
+// asks for it only where groups may form (8 score columns, one or two query
+// heads per KV head): there an item may carry a whole group of sequences and
+// items are few and long. (With 4 columns the pieces' fixed costs outweighed
+// the gain: a beam-search step took 4 % longer.) Zeroes the counters of the
+// items it splits.
+__device__ __noinline__ void plan_tail(const DecodeArgs &a, int total, int total_m,
+                                       int &tail_first, int &tail_split) {
+  const long long items_ll = (long long)total * a.num_kv_heads;
+  if (a.tail_cnt == nullptr || items_ll <= a.grid || items_ll >= INT_MAX) return;
+  const int items = static_cast<int>(items_ll);
+  const int r = items % a.grid;
+  if (r == 0) return;
+  int k = min(TAIL_MAX_SPLIT, min(a.grid / r, a.tail_slots / r));
+  const int first = items - r;
+  if (k < 2 || first < total_m * a.num_kv_heads) return;
+  const uint2 last = a.work[total - 1];  // (written before the plan's last barrier)
+  const int ls = min(static_cast<int>(last.x >> 16), a.num_seqs - 1);
+  const int tiles =
+      (last.y >> 31) != 0 ? a.grp_tiles[ls] : (static_cast<int>(last.y) + TILE - 1) / TILE;
+  k = min(k, tiles / TAIL_MIN_PIECE_TILES);
+  if (k < 2) return;
+  tail_first = first;
+  tail_split = k;
+  for (int i = threadIdx.x; i < r; i += blockDim.x) a.tail_cnt[i] = 0;
+}
+
 // Build the work list in two regions.
 //  1. Entries of several partitions: all their partitions, entry by entry,
 //     the short last partition first. Their merges then complete while the
@@ -406,13 +448,17 @@ __device__ __noinline__ void plan_small(const DecodeArgs &a, int lane) {
 // sequence's clamped length, or the leader's group word. Sequences are taken
 // in rounds of PLAN_THREADS (thread t holds sequence round*PLAN_THREADS + t),
 // so that thread order is sequence order. The merge counters are reset here
-// too.
+// too, and the tail split is decided (plan_tail).
 //
 // This grid is the programmatic dependent of what precedes it, typically the
 // previous decode call, and may start while that call is still running. It
 // waits for that grid to complete (griddepcontrol.wait) before it reads or
 // writes global memory: the context lengths may come from the kernel before
 // it, and the workspace may still be in use by the previous call.
+// TAIL: the decode kernel it feeds has the 8-column layout, which reads the
+// tail-split words (written whenever the block plans, i.e. always when groups
+// may form).
+template <bool TAIL>
 __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) {
   constexpr int NW = PLAN_THREADS / 32;
   __shared__ int wsum[NW];
@@ -609,6 +655,8 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
     __syncthreads();  // wcnt and total_m_s are rewritten by the next round
   }
   const int total = total_s;
+  int tail_first = 0, tail_split = 0;
+  if (TAIL && grouping) plan_tail(a, total, total_m, tail_first, tail_split);
   if (a.merge_cnt) {
     const int n1 = S * a.num_kv_heads * a.max_chunks;
     for (int i = tid; i < n1; i += PLAN_THREADS) a.merge_cnt[i] = 0;
@@ -617,6 +665,10 @@ __global__ void __launch_bounds__(PLAN_THREADS) plan_kernel(const DecodeArgs a) 
   if (tid == 0) {
     a.sched[0] = a.grid;  // items 0 .. grid-1 are each CTA's first, taken without the counter
     a.sched[1] = total;
+    if (TAIL) {
+      a.sched[2] = tail_first;
+      a.sched[3] = tail_split;
+    }
     if (bad_len) report(a.err, PKV_DEV_CONTEXT_LEN);
   }
 }
@@ -734,7 +786,9 @@ __device__ __forceinline__ bool consumers_all(bool v) {
 // were written by other CTAs; they are read from L2 (ld.global.cg). The
 // result goes to `out` (final), or to chunk entry `dst_idx` of the
 // second-level arrays as (o, lse). Threads tid = 0 .. nthreads-1 share it.
-template <typename T, int D>
+// BY_PIECE: the entries are pieces q0 .. q1-1 of a tail-split item in the
+// tail region (src_stride unused).
+template <typename T, int D, bool BY_PIECE = false>
 __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int G, int members,
                                          const float *src_o, const float *src_lse,
                                          int src_stride, int q0, int q1, bool final_out,
@@ -747,15 +801,20 @@ __device__ __noinline__ void merge_range(const DecodeArgs &a, int s, int h, int 
     const int cv = idx - n * V;
     const int mem = n / G;
     const size_t row = (size_t)(s + mem) * a.num_heads + h * G + (n - mem * G);
-    const float *lse = src_lse + row * src_stride + q0;
-    const float4 *po = reinterpret_cast<const float4 *>(src_o + (row * src_stride + q0) * D) + cv;
+    // Entry q of this row: a sequence row's partitions are consecutive
+    // (src_stride per row); a tail item's pieces hold TAIL_COLS rows each, the
+    // item's column n in row n of each piece.
+    const size_t base = BY_PIECE ? (size_t)q0 * TAIL_COLS + n : row * src_stride + q0;
+    constexpr size_t qs = BY_PIECE ? TAIL_COLS : 1;
+    const float *lse = src_lse + base;
+    const float4 *po = reinterpret_cast<const float4 *>(src_o + base * D) + cv;
     // All of the entries' loads are issued before the first is used.
     float lq[MERGE_CHUNK];
     float4 vq[MERGE_CHUNK];
 #pragma unroll
     for (int q = 0; q < MERGE_CHUNK; ++q) {
-      lq[q] = q < n_q ? __ldcg(lse + q) : -INFINITY;
-      vq[q] = q < n_q ? __ldcg(po + (size_t)q * V) : make_float4(0.f, 0.f, 0.f, 0.f);
+      lq[q] = q < n_q ? __ldcg(lse + q * qs) : -INFINITY;
+      vq[q] = q < n_q ? __ldcg(po + q * qs * V) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     float M = -INFINITY;
 #pragma unroll
@@ -884,7 +943,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     // list length instead of after it; it is used only if the item exists.
     const uint2 first_wk = a.work[blockIdx.x / Hkv];
     const long long list_cap = (long long)a.num_seqs * a.max_parts;
-    const int total_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
+    const int n_items = (int)min((long long)a.sched[1], list_cap) * Hkv;
+    // Tail split (see plan_kernel): items tail_first .. n_items-1 are claimed
+    // as tail_split pieces each, so claims run to total_items. (The bounds keep
+    // every piece inside the tail region whatever the words hold.)
+    int tail_first = n_items, tail_split = 1;
+    if (Shape::GROUPS && a.max_group > 1) {  // (the plan wrote the words)
+      const int f = a.sched[2], k = a.sched[3];
+      if (k >= 2 && k <= TAIL_MAX_SPLIT && f >= (int)gridDim.x && f < n_items &&
+          (long long)(n_items - f) * k <= a.tail_slots) {
+        tail_first = f;
+        tail_split = k;
+      }
+    }
+    const int total_items = tail_first + (n_items - tail_first) * tail_split;
     const int end_phase = total_items - END_ITEMS_PER_CTA * (int)gridDim.x;
     // A CTA that starts after some wait already gave up does no work. The
     // error word is loaded now and checked before the first copy is started,
@@ -914,7 +986,21 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int pk = d.kind;
         if (pk == KIND_WORK) --in_flight;
         const int np = d.nparts;
-        if (pk == KIND_WORK && np > 1) {
+        if (Shape::GROUPS && pk == KIND_WORK && d.tail >= 0) {
+          // a piece of a tail-split item: the warp that completes the item's
+          // last piece merges the pieces into `out`
+          const int j = d.tail / np;  // the item's first piece slot is j * np
+          int t = 0;
+          if (lane == 0) {
+            __threadfence();
+            t = atomicAdd(&a.tail_cnt[j], 1);
+          }
+          if (__shfl_sync(FULL_MASK, t, 0) == np - 1) {
+            (void)ld_acquire_gpu(&a.tail_cnt[j]);  // every lane: the pieces are visible
+            merge_range<T, D, true>(a, d.s, d.h, G, d.members, a.tail_o, a.tail_lse, 0, j * np,
+                                    j * np + np, true, 0, lane, 32);
+          }
+        } else if (pk == KIND_WORK && np > 1) {
           const int ms = d.s, mh = d.h, mm = d.members, ch = d.p / MERGE_CHUNK;
           const int nchunks = (np + MERGE_CHUNK - 1) / MERGE_CHUNK;
           int32_t *const cnt1 = &a.merge_cnt[(ms * Hkv + mh) * a.max_chunks + ch];
@@ -986,8 +1072,16 @@ __global__ void __launch_bounds__(THREADS, 2)
       // Items are entry-major: the KV heads of one entry are consecutive items.
       // A block's heads are contiguous in the pool, so CTAs working on
       // neighbouring items read neighbouring 4 KB slices (open DRAM rows).
-      const uint2 wk = first_post ? first_wk : a.work[item / Hkv];  // first_post: item == blockIdx.x
-      const int h = item - (item / Hkv) * Hkv;
+      // A claim past tail_first is piece `piece` of item `wi` (its pieces are
+      // consecutive claims, so they run side by side).
+      int wi = item, piece = -1;
+      if (Shape::GROUPS && item >= tail_first) {
+        const int jj = item - tail_first;
+        wi = tail_first + jj / tail_split;
+        piece = jj - (jj / tail_split) * tail_split;
+      }
+      const uint2 wk = first_post ? first_wk : a.work[wi / Hkv];  // first_post: item == blockIdx.x
+      const int h = wi - (wi / Hkv) * Hkv;
       const int s = min(static_cast<int>(wk.x >> 16), a.num_seqs - 1);
       const int p = static_cast<int>(wk.x & 0xffffu);
       // One sequence (its clamped length in the entry), or a shared-prefix
@@ -1022,8 +1116,11 @@ __global__ void __launch_bounds__(THREADS, 2)
         own_lo = sh + own_incl - own_n;
         tiles = sh + __shfl_sync(FULL_MASK, own_incl, 31);
       }
-      const int ptg = group_part_tiles(a, grouped, tiles);
-      const int tile0 = p * ptg;
+      // a tail piece: its share of the item's tiles (the plan split only
+      // one-partition items)
+      const int ptg = piece >= 0 ? max(1, (tiles + tail_split - 1) / tail_split)
+                                 : group_part_tiles(a, grouped, tiles);
+      const int tile0 = (piece >= 0 ? piece : p) * ptg;
       const int n_tiles = max(0, min(tiles, tile0 + ptg) - tile0);
       if (first_post) {
         first_post = false;
@@ -1114,10 +1211,11 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (lane == 0) {
         d.kind = KIND_WORK;
         d.s = s;
-        d.p = p;
+        d.p = piece >= 0 ? piece : p;
         d.h = h;
         d.n_tiles = n_tiles;
-        d.nparts = (tiles + ptg - 1) / ptg;
+        d.nparts = piece >= 0 ? tail_split : (tiles + ptg - 1) / ptg;
+        if constexpr (Shape::GROUPS) d.tail = piece >= 0 ? item - tail_first : -1;
         d.members = members;
         d.tile0 = tile0;
         d.sh = sh;
@@ -1273,7 +1371,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       continue;
     }
     const int s = dref.s, p = dref.p, h = dref.h, n_tiles = dref.n_tiles;
-    const int nparts = dref.nparts;
+    const int nparts = dref.nparts, tail = Shape::GROUPS ? dref.tail : -1;
     const int members = dref.members, tile0 = dref.tile0;
     const bool one_seq = !Shape::GROUPS || members == 1;
     const int ncol = members * G;  // head rows attended: G per member
@@ -1583,22 +1681,35 @@ __global__ void __launch_bounds__(THREADS, 2)
       scales[NH * NCW + n] = den > 0.f ? M + lg2_approx(den) : -INFINITY;
     }
     consumers_sync();
-    // 3) outputs
-    const bool single = nparts <= 1;
-    for (int idx = threadIdx.x; idx < ncol * D; idx += NCW * 32) {
-      const int n = idx / D;
-      const int dd = idx - n * D;
+    // 3) outputs: element dd of column n's combined row
+    auto combined = [&](int n, int dd) {
       float o = 0.f;
 #pragma unroll
       for (int w = 0; w < NCW; ++w)
         if (area[w]) o += scales[n * NCW + w] * area[w][n * AS + dd];
-      const int mem = n / G;  // row n is query head h*G + n%G of member mem
-      const size_t row = (size_t)(s + mem) * Hq + h * G + (n - mem * G);
-      if (single) {
-        out[row * D + dd] = from_float<T>(o);
-      } else {
-        a.ws_o[(row * a.max_parts + p) * D + dd] = o;
-        if (dd == 0) a.ws_lse[row * a.max_parts + p] = scales[NH * NCW + n];
+      return o;
+    };
+    if (tail >= 0) {  // a tail piece: column n goes to row n of its slot
+      for (int idx = threadIdx.x; idx < ncol * D; idx += NCW * 32) {
+        const int n = idx / D;
+        const int dd = idx - n * D;
+        a.tail_o[((size_t)tail * TAIL_COLS + n) * D + dd] = combined(n, dd);
+        if (dd == 0) a.tail_lse[(size_t)tail * TAIL_COLS + n] = scales[NH * NCW + n];
+      }
+    } else {
+      const bool single = nparts <= 1;
+      for (int idx = threadIdx.x; idx < ncol * D; idx += NCW * 32) {
+        const int n = idx / D;
+        const int dd = idx - n * D;
+        const float o = combined(n, dd);
+        const int mem = n / G;  // row n is query head h*G + n%G of member mem
+        const size_t row = (size_t)(s + mem) * Hq + h * G + (n - mem * G);
+        if (single) {
+          out[row * D + dd] = from_float<T>(o);
+        } else {
+          a.ws_o[(row * a.max_parts + p) * D + dd] = o;
+          if (dd == 0) a.ws_lse[row * a.max_parts + p] = scales[NH * NCW + n];
+        }
       }
     }
     // This warp is done with the item's descriptor and q rows. Its arrival
@@ -1663,7 +1774,7 @@ cudaError_t launch_tc(const DecodeArgs &a, const CUtensorMap &tmK, const CUtenso
   pcfg.stream = stream;
   pcfg.attrs = attr;
   pcfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&pcfg, plan_kernel, b);
+  e = cudaLaunchKernelEx(&pcfg, plan_kernel<Shape::GROUPS>, b);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);

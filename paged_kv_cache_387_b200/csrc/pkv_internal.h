@@ -36,7 +36,8 @@ struct DecodeArgs {
   // Work list of the persistent decode kernel (written by the plan kernel):
   uint2 *work;         // [<= S*max_parts] {seq << 16 | partition, context length, or
                        //  1 << 31 | the leader's grp word for a group}
-  int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries
+  int32_t *sched;      // [0] dispatch counter, [1] number of work-list entries,
+                       // [2] first tail item, [3] pieces per tail item (< 2: none)
   // Partition merging (split contexts). Partitions are merged in chunks of
   // MERGE_CHUNK; a context with more than one chunk is merged in two levels.
   int32_t *merge_cnt;  // [S*Hkv][max_chunks] finished partitions per chunk; zeroed by the plan
@@ -54,9 +55,24 @@ struct DecodeArgs {
                        // that may sit in different blocks
   int wave_clusters;   // single-wave kernel: clusters per (sequence, KV head); above 1 each
                        // writes its merged partitions to a workspace slot (0 or 1: one)
+  // Tail split of the persistent decode (see plan_kernel): the last items of
+  // the work list are each attended as several pieces, merged when the last
+  // piece of an item finishes.
+  float *tail_o;       // [tail_slots][TAIL_COLS][D] piece outputs (normalised)
+  float *tail_lse;     // [tail_slots][TAIL_COLS] piece log2-sum-exp
+  int32_t *tail_cnt;   // [tail_slots] finished pieces per tail item; zeroed by the plan
+  int tail_slots;      // pieces the tail region holds
 };
 
 constexpr int MERGE_CHUNK = 16;  // partitions merged together at the first level
+
+// Tail split: a piece holds up to TAIL_COLS query-head rows (one work item's
+// score columns); at most TAIL_MAX_PIECES pieces per call, TAIL_MAX_SPLIT per
+// item, and each piece spans at least TAIL_MIN_PIECE_TILES 16-token tiles.
+constexpr int TAIL_COLS = 8;
+constexpr int TAIL_MAX_PIECES = 512;
+constexpr int TAIL_MAX_SPLIT = 8;
+constexpr int TAIL_MIN_PIECE_TILES = 8;
 
 // Single-wave decode (decode_wave.cu): at most this many partitions per
 // (sequence, KV head), one thread-block cluster of that many CTAs.
@@ -77,13 +93,16 @@ constexpr int WAVE_SPLIT_MIN_GAIN = 16;
 constexpr int WAVE_MAX_WARP_CHAIN = 64;
 
 // Decode workspace, in order: scheduling words (256 B), the work list, the
-// per-sequence group words (two int32 per sequence), then
-// (only when a context can span several partitions) the merge counters, the
-// partition outputs with their log2-sum-exp values, and (only when a context
-// can span several merge chunks) the chunk results. Each region is 256-byte
-// aligned.
+// per-sequence group words (two int32 per sequence), then (only when a
+// context can span several partitions) the merge counters, the partition
+// outputs with their log2-sum-exp values, and (only when a context can span
+// several merge chunks) the chunk results, and last the tail-split region
+// (piece counters, outputs and log2-sum-exp values of min(TAIL_MAX_PIECES,
+// S * Hq * max_parts) pieces). Each region is 256-byte aligned.
 struct WorkspaceLayout {
-  size_t sched_off, work_off, grp_off, cnt_off, cnt2_off, o_off, lse_off, o2_off, lse2_off, total;
+  size_t sched_off, work_off, grp_off, tcnt_off, to_off, tlse_off, cnt_off, cnt2_off, o_off,
+      lse_off, o2_off, lse2_off, total;
+  long long tail_slots;
 };
 WorkspaceLayout workspace_layout(long long S, long long Hq, long long D, long long max_parts);
 

@@ -58,6 +58,8 @@ def test_workspace_arithmetic(lib):
     def expected(S, Hq, D, L, P):
         parts = 1 if P == 0 else -(-max(L, 1) // P)  # partitions of the longest context
         total = 256 + rnd(S * parts * 8) + rnd(2 * S * 4)  # sched words, work list, group words
+        pieces = min(512, S * Hq * parts)                    # tail split: counters, 8 rows each
+        total += rnd(pieces * 4) + rnd(pieces * 8 * D * 4) + rnd(pieces * 8 * 4)
         if parts > 1:
             chunks = -(-parts // 16)
             total += (rnd(S * Hq * chunks * 4) + rnd(S * Hq * 4)      # merge counters
@@ -66,20 +68,30 @@ def test_workspace_arithmetic(lib):
                 total += rnd(S * Hq * chunks * D * 4) + rnd(S * Hq * chunks * 4)
         return total
 
+    # tail-split region: min(512, S*Hq*partitions) pieces, each a counter, 8
+    # fp32 output rows and 8 fp32 log2-sum-exp values
+    def tail(S, Hq, D, parts):
+        n = min(512, S * Hq * parts)
+        return rnd(n * 4) + rnd(n * 8 * D * 4) + rnd(n * 8 * 4)
+
+    assert tail(8, 32, 128, 1) == 1024 + 256 * 8 * 128 * 4 + 256 * 8 * 4
+    assert tail(100, 8, 64, 1) == 2048 + 512 * 8 * 64 * 4 + 512 * 8 * 4  # capped at 512
     # scheduling words (256 B) + work list (8 bytes per (seq, partition)) +
     # shared-prefix group words (two int32 per sequence), each region rounded
     # up to 256 B
-    assert f(8, 32, 128, 512, 512) == 256 + 256 + 256   # one partition: no partials
-    assert f(8, 32, 128, 100, 0) == 256 + 256 + 256     # unsplit
-    assert f(100, 8, 64, 100, 0) == 256 + rnd(100 * 8) + rnd(100 * 8)
+    assert f(8, 32, 128, 512, 512) == 256 + 256 + 256 + tail(8, 32, 128, 1)  # no partials
+    assert f(8, 32, 128, 100, 0) == 256 + 256 + 256 + tail(8, 32, 128, 1)    # unsplit
+    assert f(100, 8, 64, 100, 0) == 256 + rnd(100 * 8) + rnd(100 * 8) + tail(100, 8, 64, 1)
     # 8 seqs x 32 heads x 256 partitions (16 merge chunks of 16): chunk and
     # final merge counters, fp32 partition outputs + lse, chunk results + lse
     S, Hq, D, P, C = 8, 32, 128, 256, 16
-    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + 256 + S * Hq * C * 4 + S * Hq * 4
+    assert f(S, Hq, D, 131072, 512) == (256 + S * P * 8 + 256 + tail(S, Hq, D, P)
+                                        + S * Hq * C * 4 + S * Hq * 4
                                         + S * Hq * P * D * 4 + S * Hq * P * 4
                                         + S * Hq * C * D * 4 + S * Hq * C * 4)
     # 33 tokens in 16-token partitions = 3 partitions, one merge chunk
-    assert f(1, 1, 64, 33, 16) == 256 + 256 + 256 + 256 + 256 + 3 * 64 * 4 + 256
+    assert f(1, 1, 64, 33, 16) == (256 + 256 + 256 + tail(1, 1, 64, 3)
+                                   + 256 + 256 + 3 * 64 * 4 + 256)
     for args in [(100, 8, 64, 100, 0), (3, 40, 128, 1064, 2048), (256, 32, 128, 4096, 2048),
                  (5, 2, 64, 20000, 16)]:
         assert f(*args) == expected(*args), args
