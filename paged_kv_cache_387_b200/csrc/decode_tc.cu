@@ -1510,16 +1510,41 @@ __global__ void __launch_bounds__(THREADS, 2)
         __syncwarp();
       }
 
-      // ---- scores: S^T = K . Q^T (two independent accumulation chains) ----
+      // ---- scores: S^T = K . Q^T in independent accumulation chains: two
+      // (sa, sb), and with 4 columns two more (sc, sd) for the odd k-chunks.
+      // (Four chains in the 8-column layout measured 5-6 % slower.) ----
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (Shape::GROUPS) {
 #pragma unroll
-      for (int jj = 0; jj < D / 32; ++jj) {
-        const int Lc = (jj >> 1) * 8 + 2 * c + (jj & 1);
-        const uint32_t rowg = ks + (Lc >> 3) * HALF_BYTES + g * 128 + (((Lc & 7) ^ g) << 4);
-        const uint4 ka = lds128(rowg);            // token g
-        const uint4 kb = lds128(rowg + 8 * 128);  // token g + 8 (same swizzle phase)
-        mma16816<T>(sa, ka.x, kb.x, ka.y, kb.y, qf[jj].x, qf[jj].y);
-        mma16816<T>(sb, ka.z, kb.z, ka.w, kb.w, qf[jj].z, qf[jj].w);
+        for (int jj = 0; jj < D / 32; ++jj) {
+          const int Lc = (jj >> 1) * 8 + 2 * c + (jj & 1);
+          const uint32_t rowg = ks + (Lc >> 3) * HALF_BYTES + g * 128 + (((Lc & 7) ^ g) << 4);
+          const uint4 ka = lds128(rowg);            // token g
+          const uint4 kb = lds128(rowg + 8 * 128);  // token g + 8 (same swizzle phase)
+          mma16816<T>(sa, ka.x, kb.x, ka.y, kb.y, qf[jj].x, qf[jj].y);
+          mma16816<T>(sb, ka.z, kb.z, ka.w, kb.w, qf[jj].z, qf[jj].w);
+        }
+      } else {
+        float sc[4] = {0.f, 0.f, 0.f, 0.f}, sd[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int jj = 0; jj < D / 32; ++jj) {
+          const int Lc = (jj >> 1) * 8 + 2 * c + (jj & 1);
+          const uint32_t rowg = ks + (Lc >> 3) * HALF_BYTES + g * 128 + (((Lc & 7) ^ g) << 4);
+          const uint4 ka = lds128(rowg);            // token g
+          const uint4 kb = lds128(rowg + 8 * 128);  // token g + 8 (same swizzle phase)
+          if (jj & 1) {
+            mma16816<T>(sc, ka.x, kb.x, ka.y, kb.y, qf[jj].x, qf[jj].y);
+            mma16816<T>(sd, ka.z, kb.z, ka.w, kb.w, qf[jj].z, qf[jj].w);
+          } else {
+            mma16816<T>(sa, ka.x, kb.x, ka.y, kb.y, qf[jj].x, qf[jj].y);
+            mma16816<T>(sb, ka.z, kb.z, ka.w, kb.w, qf[jj].z, qf[jj].w);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          sa[r] += sc[r];
+          sb[r] += sd[r];
+        }
       }
 
       // ---- online softmax (heads 2c, 2c+1; tokens g, g+8) ----
