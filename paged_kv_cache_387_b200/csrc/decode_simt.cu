@@ -1,12 +1,15 @@
 // Paged decode attention for fp32 inputs, and the split-context merge.
 //
 // fp32 inputs keep fp32 arithmetic end to end: no tensor-core rounding of K,
-// V or P. One CTA (4 warps) attends one (sequence, query head, partition).
-// Each warp walks every 4th token: it looks up the token's physical block in
-// the block table, forms the score with a warp-wide dot product and updates a
-// running max / sum / output. That is the online walk of page "PagedAttention
-// Analysis" (ryotta.opik.net), section 3, one token at a time. The warps are
-// then combined in shared memory.
+// V or P. One CTA (4 warps) attends one (sequence, KV head, partition) for up
+// to SIMT_GMAX of the query heads that share the KV head (a group of more is
+// split over several CTAs). Each warp walks every 4th token: it looks up the
+// token's physical block in the block table, loads the token's K and V rows
+// once (one vector per lane) for all its heads, forms each head's score with
+// a warp-wide dot product and updates that head's running max / sum /
+// output. That is the online walk of page "PagedAttention Analysis"
+// (ryotta.opik.net), section 3, one token at a time. The warps are then
+// combined in shared memory, head by head.
 //
 // The merge kernel combines the partitions of a split context. Partition p
 // contributes its normalised output o_p with weight 2^(lse_p - lse), where
@@ -18,31 +21,51 @@ namespace pkv {
 namespace {
 
 constexpr int SIMT_WARPS = 4;
+constexpr int SIMT_GMAX = 8;  // query heads one CTA attends together
+
+// E consecutive floats (E = 2 or 4) as one aligned vector load.
+template <int E>
+__device__ __forceinline__ void load_vec(const float *p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    v[0] = t.x;
+    v[1] = t.y;
+    v[2] = t.z;
+    v[3] = t.w;
+  } else {
+    static_assert(E == 2, "head_dim 64 or 128");
+    const float2 t = *reinterpret_cast<const float2 *>(p);
+    v[0] = t.x;
+    v[1] = t.y;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(SIMT_WARPS * 32) decode_simt_f32_kernel(const DecodeArgs a) {
   constexpr int E = D / 32;  // elements per lane
-  __shared__ float red_acc[SIMT_WARPS][D];
-  __shared__ float red_ml[SIMT_WARPS][2];
+  __shared__ float red_acc[SIMT_WARPS][SIMT_GMAX][D];
+  __shared__ float red_ml[SIMT_WARPS][SIMT_GMAX][2];
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int p = blockIdx.x;
-  const int hq = blockIdx.y;
   const int s = blockIdx.z;
   const int Hq = a.num_heads;
   const int Hkv = a.num_kv_heads;
   const int G = Hq / Hkv;
-  const int kvh = hq / G;
+  const int nchunk = (G + SIMT_GMAX - 1) / SIMT_GMAX;  // CTAs per KV head
+  const int kvh = blockIdx.y / nchunk;
+  const int h0 = kvh * G + (blockIdx.y - kvh * nchunk) * SIMT_GMAX;  // first query head
+  const int ng = min(SIMT_GMAX, kvh * G + G - h0);                   // heads of this CTA
   const int B = a.block_size;
 
   const int L = effective_len(a.context_lens[s], a.max_context_len, a.max_blocks, B,
                               threadIdx.x == 0 ? a.err : nullptr);
   float *out = static_cast<float *>(a.out);
-  const size_t row = (size_t)s * Hq + hq;
+  const size_t row0 = (size_t)s * Hq + h0;  // row of head h0; head h0 + g is row0 + g
   if (L <= 0) {
     if (p == 0)
-      for (int d = threadIdx.x; d < D; d += SIMT_WARPS * 32) out[row * D + d] = 0.f;
+      for (int i = threadIdx.x; i < ng * D; i += SIMT_WARPS * 32) out[row0 * D + i] = 0.f;
     return;
   }
   const int t_begin = p * a.part_tokens;
@@ -50,18 +73,30 @@ __global__ void __launch_bounds__(SIMT_WARPS * 32) decode_simt_f32_kernel(const 
   const int t_end = min(L, t_begin + a.part_tokens);
   const int nparts = (L + a.part_tokens - 1) / a.part_tokens;
 
-  const float *qrow = static_cast<const float *>(a.q) + row * D;
-  float qv[E];
+  const float *q = static_cast<const float *>(a.q);
+  float qv[SIMT_GMAX][E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) qv[e] = qrow[lane * E + e];
+  for (int g = 0; g < SIMT_GMAX; ++g) {
+    if (g < ng) {
+      load_vec<E>(q + (row0 + g) * D + lane * E, qv[g]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) qv[g][e] = 0.f;
+    }
+  }
 
   const float *kp = static_cast<const float *>(a.k_pool);
   const float *vp = static_cast<const float *>(a.v_pool);
   const int32_t *bt = a.block_tables + (size_t)s * a.max_blocks;
 
-  float m = -INFINITY, l = 0.f, acc[E];
+  float m[SIMT_GMAX], l[SIMT_GMAX], acc[SIMT_GMAX][E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  for (int g = 0; g < SIMT_GMAX; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[g][e] = 0.f;
+  }
 
   for (int t = t_begin + warp; t < t_end; t += SIMT_WARPS) {
     const int phys = bt[t / B];
@@ -70,43 +105,64 @@ __global__ void __launch_bounds__(SIMT_WARPS * 32) decode_simt_f32_kernel(const 
       continue;
     }
     const size_t base = (((size_t)phys * Hkv + kvh) * B + (t % B)) * D + lane * E;
-    float dot = 0.f;
+    float kv[E], vv[E];
+    load_vec<E>(kp + base, kv);
+    load_vec<E>(vp + base, vv);
+    float dot[SIMT_GMAX];
 #pragma unroll
-    for (int e = 0; e < E; ++e) dot = fmaf(qv[e], kp[base + e], dot);
+    for (int g = 0; g < SIMT_GMAX; ++g) {
+      dot[g] = 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(FULL_MASK, dot, off);
-    const float x = dot * a.scale_log2;
-    const float mn = fmaxf(m, x);
-    const float al = exp2f(m - mn);
-    const float pr = exp2f(x - mn);
-    l = l * al + pr;
+      for (int e = 0; e < E; ++e) dot[g] = fmaf(qv[g][e], kv[e], dot[g]);
+    }
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = fmaf(pr, vp[base + e], acc[e] * al);
-    m = mn;
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+      for (int g = 0; g < SIMT_GMAX; ++g)
+        if (g < ng) dot[g] += __shfl_xor_sync(FULL_MASK, dot[g], off);
+#pragma unroll
+    for (int g = 0; g < SIMT_GMAX; ++g) {
+      if (g >= ng) continue;
+      const float x = dot[g] * a.scale_log2;
+      const float mn = fmaxf(m[g], x);
+      const float al = exp2f(m[g] - mn);
+      const float pr = exp2f(x - mn);
+      l[g] = l[g] * al + pr;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[g][e] = fmaf(pr, vv[e], acc[g][e] * al);
+      m[g] = mn;
+    }
   }
 
 #pragma unroll
-  for (int e = 0; e < E; ++e) red_acc[warp][lane * E + e] = acc[e];
-  if (lane == 0) {
-    red_ml[warp][0] = m;
-    red_ml[warp][1] = l;
+  for (int g = 0; g < SIMT_GMAX; ++g) {
+    if (g >= ng) continue;
+#pragma unroll
+    for (int e = 0; e < E; ++e) red_acc[warp][g][lane * E + e] = acc[g][e];
+    if (lane == 0) {
+      red_ml[warp][g][0] = m[g];
+      red_ml[warp][g][1] = l[g];
+    }
   }
   __syncthreads();
 
-  for (int d = threadIdx.x; d < D; d += SIMT_WARPS * 32) {
+  for (int i = threadIdx.x; i < ng * D; i += SIMT_WARPS * 32) {
+    const int g = i / D;
+    const int d = i - g * D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < SIMT_WARPS; ++w) M = fmaxf(M, red_ml[w][0]);
+    for (int w = 0; w < SIMT_WARPS; ++w) M = fmaxf(M, red_ml[w][g][0]);
     float num = 0.f, den = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < SIMT_WARPS; ++w) {
-        const float f = exp2f(red_ml[w][0] - M);
-        num += f * red_acc[w][d];
-        den += f * red_ml[w][1];
+        const float f = exp2f(red_ml[w][g][0] - M);
+        num += f * red_acc[w][g][d];
+        den += f * red_ml[w][g][1];
       }
     }
     const float o = den > 0.f ? num / den : 0.f;
+    const size_t row = row0 + g;
     if (nparts == 1) {
       out[row * D + d] = o;
     } else {
@@ -213,7 +269,8 @@ cudaError_t launch_merge_t(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_decode_simt_f32(const DecodeArgs &a, cudaStream_t stream) {
-  dim3 grid(a.max_parts, a.num_heads, a.num_seqs);
+  const int G = a.num_heads / a.num_kv_heads;
+  dim3 grid(a.max_parts, a.num_kv_heads * ((G + SIMT_GMAX - 1) / SIMT_GMAX), a.num_seqs);
   if (a.head_dim == 64)
     decode_simt_f32_kernel<64><<<grid, SIMT_WARPS * 32, 0, stream>>>(a);
   else
