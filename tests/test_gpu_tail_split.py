@@ -130,21 +130,23 @@ def test_three_or_more_heads_per_kv_head_are_not_split(Hq, Hkv):
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 8)])  # G = 1 (8 members), G = 2 (4 members)
+@pytest.mark.parametrize("D,B,dt", [(128, 16, torch.float16), (64, 24, torch.bfloat16)])
 @pytest.mark.parametrize("fused", [False, True])
-def test_shared_prefix_group_items(Hq, Hkv, fused):
+def test_shared_prefix_group_items(Hq, Hkv, D, B, dt, fused):
     """Groups of samples that share a prompt: the tail's group items are split,
-    each piece covering part of the shared tiles or of the members' own ones."""
+    each piece covering part of the shared tiles or of the members' own ones.
+    Block 24 puts the two 8-token halves of some tiles in different blocks."""
     members = 8 // (Hq // Hkv)
     n_groups = (grid_ctas() + 24) // Hkv
-    rng = np.random.default_rng(5 + Hq)
+    rng = np.random.default_rng(5 + Hq + B)
     groups = [(int(rng.integers(400, 700)), [int(x) for x in rng.integers(1, 80, size=members)])
               for _ in range(n_groups)]
-    c = make_sharing_case("tailg", Hq, Hkv, 128, 16, groups, torch.float16, seed=21 + Hq,
-                          device=DEV, with_append=True)
+    c = make_sharing_case("tailg", Hq, Hkv, D, B, groups, dt, seed=21 + Hq + B, device=DEV,
+                          with_append=True)
     out, ref, words = run(c, 2048, fused)
     assert words[3] >= 2, words  # the tail was split
     assert words[2] == n_groups * Hkv - n_groups * Hkv % grid_ctas()
-    assert_close_to_oracle(out, ref, torch.float16, f"tail split groups G{Hq // Hkv}")
+    assert_close_to_oracle(out, ref, dt, f"tail split groups G{Hq // Hkv} D{D} B{B}")
 
 
 def test_remainder_too_large_is_not_split():
