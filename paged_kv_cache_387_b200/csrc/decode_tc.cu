@@ -38,7 +38,9 @@
 //   fetch-and-add on its chunk's counter). The scheduler warp that completes a
 //   chunk of 16 partitions merges it right away, and the one that completes
 //   the last chunk merges the chunks into `out`: the merges never queue behind
-//   work items in a descriptor ring. No CTA ever waits for another.
+//   work items in a descriptor ring. The pieces of a tail-split item are
+//   counted the same way, and the warp that completes the last piece merges
+//   them. No CTA ever waits for another.
 //   Warps 0-3 are consumers. Each owns a ring of stages in shared memory and
 //   takes tiles w, w+4, w+8, ... of every item. Its lane 0 fills the ring
 //   with TMA, completing on the stage's mbarrier:
